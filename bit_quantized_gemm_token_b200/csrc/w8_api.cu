@@ -1,0 +1,263 @@
+// w8_api.cu -- the C ABI (include/w8.h): argument validation, device check, variant
+// resolution (per-shape table, then a built-in rule) and dispatch to the kernels.
+// Nothing here allocates device memory or synchronises.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "w8_internal.h"
+
+namespace w8 {
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct DevInfo {
+    bool probed = false;
+    bool ok = false;
+    int sms = 0;
+};
+
+std::mutex g_dev_mu;
+DevInfo g_dev[64];
+
+// ---- per-shape table ----------------------------------------------------------------
+struct Entry {
+    int fmt, N, K, m_max, variant;
+};
+std::mutex g_tab_mu;
+std::vector<Entry> g_table;
+
+}  // namespace
+
+int check_device(int* sm_count)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return W8_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo& d = g_dev[dev];
+    if (!d.probed) {
+        d.probed = true;
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess) {
+            d.ok = (major == 10 && minor == 0);
+            d.sms = sms;
+        }
+    }
+    if (!d.ok) return W8_ERR_NO_DEVICE;
+    if (sm_count) *sm_count = d.sms;
+    return W8_OK;
+}
+
+int table_lookup(int fmt, int N, int K, int M)
+{
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    const Entry* best = nullptr;
+    for (const Entry& e : g_table)
+        if (e.fmt == fmt && e.N == N && e.K == K && e.m_max >= M && (!best || e.m_max < best->m_max)) best = &e;
+    return best ? best->variant : 0;
+}
+
+namespace {
+
+// Built-in rule when the table has no entry: Swap-AB with the narrowest token tile for
+// decode-sized M, the Standard 128 x 128 tile otherwise; always the balanced partition
+// (weights are streamed evenly by every SM; the partial-sum traffic stays in L2).
+int builtin_variant(int fmt, int M)
+{
+    const bool block = fmt >= W8_FMT_BLOCK_FP8;
+    if (M <= 16) return W8_VARIANT(1, 0, kTileBN16, 1);
+    if (M <= 32) return W8_VARIANT(1, 0, kTileBN32, 1);
+    if (M <= 64) return W8_VARIANT(1, 0, kTileBN64, 1);
+    return W8_VARIANT(0, 0, block ? kTileBN64 : kTileBN128, 1);
+}
+
+int resolve(int fmt, int M, int N, int K, int variant, int sms, GemmPlan* plan)
+{
+    int v = variant;
+    if (!(v & W8_V_EXPLICIT)) {
+        const int pdl = v & W8_V_PDL;   // AUTO may still ask for PDL
+        v = table_lookup(fmt, N, K, M);
+        if (!v) v = builtin_variant(fmt, M);
+        v |= pdl;
+    }
+    const int rc = gemm_plan(fmt, M, N, K, v, sms, plan);
+    return rc == W8_OK ? v : rc;
+}
+
+int gemm_common(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale, void* out,
+                int32_t* out_i32, int M, int N, int K, int variant, void* workspace, size_t ws_bytes,
+                cudaStream_t s)
+{
+    if (!A_q || !W_q || (!out && !out_i32)) return W8_ERR_INVALID_ARG;
+    if (!out_i32 && (!A_scale || !W_scale)) return W8_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0) return W8_ERR_INVALID_ARG;
+    if (!aligned(A_q, 16) || !aligned(W_q, 16)) return W8_ERR_ALIGNMENT;
+    if (out && !aligned(out, 2)) return W8_ERR_ALIGNMENT;
+    if (out_i32 && !aligned(out_i32, 4)) return W8_ERR_ALIGNMENT;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != W8_OK) return rc;
+    GemmPlan plan;
+    rc = resolve(fmt, M, N, K, variant, sms, &plan);
+    if (rc < 0) return rc;
+    return gemm_launch(plan, A_q, A_scale, W_q, W_scale, out, out_i32, workspace, ws_bytes, s);
+}
+
+bool row_args_ok(const void* x, int M, int K, int ldx, const void* q, const float* scale)
+{
+    return x && q && scale && M > 0 && K > 0 && ldx >= K;
+}
+
+}  // namespace
+}  // namespace w8
+
+using namespace w8;
+
+extern "C" {
+
+int w8_quant_per_token(int qfmt, const void* x, int M, int K, int ldx, void* q, float* scale, int group, int ue8m0,
+                       w8_stream_t stream)
+{
+    if (!row_args_ok(x, M, K, ldx, q, scale)) return W8_ERR_INVALID_ARG;
+    if (qfmt != W8_Q_FP8 && qfmt != W8_Q_INT8) return W8_ERR_INVALID_ARG;
+    if (group != 0 && group != 128) return W8_ERR_UNSUPPORTED;
+    if ((group != 0 || ue8m0) && qfmt != W8_Q_FP8) return W8_ERR_UNSUPPORTED;
+    if (ue8m0 && group == 0) return W8_ERR_UNSUPPORTED;
+    if (K % 8 != 0 || ldx % 8 != 0 || !aligned(x, 16) || !aligned(q, 8) || !aligned(scale, 4))
+        return W8_ERR_ALIGNMENT;
+    if (group != 0 && K % group != 0) return W8_ERR_UNSUPPORTED;
+    if (group == 0 && K > kRowMaxK) return W8_ERR_UNSUPPORTED;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (group == 0) return launch_quant_rows(qfmt, x, M, K, ldx, q, scale, s);
+    return launch_quant_group128(x, M, K, ldx, q, scale, ue8m0, s);
+}
+
+int w8_quant_weight_block(const void* w, int N, int K, void* q, float* scale, int ue8m0, w8_stream_t stream)
+{
+    if (!w || !q || !scale || N <= 0 || K <= 0) return W8_ERR_INVALID_ARG;
+    if (K % 8 != 0 || !aligned(w, 16) || !aligned(q, 8) || !aligned(scale, 4)) return W8_ERR_ALIGNMENT;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    return launch_quant_weight_block(w, N, K, q, scale, ue8m0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, int ldx, void* q, float* scale,
+                     w8_stream_t stream)
+{
+    if (!row_args_ok(x, M, H, ldx, q, scale) || !gamma) return W8_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f)) return W8_ERR_INVALID_ARG;
+    if (H % 8 != 0 || ldx % 8 != 0 || !aligned(x, 16) || !aligned(gamma, 16) || !aligned(q, 8) || !aligned(scale, 4))
+        return W8_ERR_ALIGNMENT;
+    if (H > kRowMaxK) return W8_ERR_UNSUPPORTED;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    return launch_rmsnorm_quant(x, gamma, eps, M, H, ldx, q, scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_silu_mul_quant(const void* gate_up, int M, int I, int ld, void* q, float* scale, w8_stream_t stream)
+{
+    if (!gate_up || !q || !scale || M <= 0 || I <= 0 || ld < 2 * I) return W8_ERR_INVALID_ARG;
+    if (I % 8 != 0 || ld % 8 != 0 || !aligned(gate_up, 16) || !aligned(q, 8) || !aligned(scale, 4))
+        return W8_ERR_ALIGNMENT;
+    if (I > kRowMaxK) return W8_ERR_UNSUPPORTED;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    return launch_silu_mul_quant(gate_up, M, I, ld, q, scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale, void* out, int M,
+            int N, int K, int variant, void* workspace, size_t ws_bytes, w8_stream_t stream)
+{
+    if (!out) return W8_ERR_INVALID_ARG;
+    return gemm_common(fmt, A_q, A_scale, W_q, W_scale, out, nullptr, M, N, K, variant, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int N, int K, int variant,
+                      void* workspace, size_t ws_bytes, w8_stream_t stream)
+{
+    if (!acc) return W8_ERR_INVALID_ARG;
+    return gemm_common(W8_FMT_INT8, A_q, nullptr, W_q, nullptr, nullptr, acc, M, N, K, variant, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant)
+{
+    int sms = 0;
+    if (check_device(&sms) != W8_OK) sms = 148;   // planning only: usable without a device
+    GemmPlan plan;
+    return resolve(fmt, M, N, K, variant, sms, &plan);
+}
+
+size_t w8_gemm_workspace_size(int fmt, int M, int N, int K, int variant)
+{
+    int sms = 0;
+    if (check_device(&sms) != W8_OK) sms = 148;
+    GemmPlan plan;
+    if (resolve(fmt, M, N, K, variant, sms, &plan) < 0) return (size_t)-1;
+    return plan.ws_bytes;
+}
+
+int w8_load_table(const char* path)
+{
+    if (!path) return W8_ERR_INVALID_ARG;
+    FILE* f = std::fopen(path, "r");
+    if (!f) return W8_ERR_IO;
+    std::vector<Entry> t;
+    char line[512];
+    bool bad = false;
+    while (std::fgets(line, sizeof line, f)) {
+        char* hash = std::strchr(line, '#');
+        if (hash) *hash = 0;
+        Entry e;
+        unsigned v = 0;
+        char extra[4];
+        int n = std::sscanf(line, "%d %d %d %d %x %3s", &e.fmt, &e.N, &e.K, &e.m_max, &v, extra);
+        if (n <= 0) continue;   // blank or comment
+        if (n != 5 || e.fmt < 0 || e.fmt > 3 || e.N <= 0 || e.K <= 0 || e.m_max <= 0 || !(v & W8_V_EXPLICIT)) {
+            bad = true;
+            break;
+        }
+        e.variant = (int)v;
+        t.push_back(e);
+    }
+    std::fclose(f);
+    if (bad) return W8_ERR_IO;
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    g_table.swap(t);
+    return (int)g_table.size();
+}
+
+void w8_clear_table(void)
+{
+    std::lock_guard<std::mutex> lk(g_tab_mu);
+    g_table.clear();
+}
+
+int w8_device_status(int clear) { return gemm_device_status(clear); }
+
+const char* w8_status_string(int status)
+{
+    switch (status) {
+    case W8_OK: return "ok";
+    case W8_ERR_INVALID_ARG: return "invalid argument";
+    case W8_ERR_UNSUPPORTED: return "unsupported format, variant or size";
+    case W8_ERR_ALIGNMENT: return "misaligned pointer, stride or size";
+    case W8_ERR_WORKSPACE: return "workspace missing or too small";
+    case W8_ERR_CUDA: return "CUDA runtime error";
+    case W8_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case W8_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    case W8_ERR_IO: return "table file missing or malformed";
+    default: return "unknown status";
+    }
+}
+
+int w8_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// w8_internal.h -- declarations shared by the library's translation units (not part of
+// the public ABI, which is include/w8.h).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/w8.h"
+
+namespace w8 {
+
+// ---- device / launch helpers (w8_api.cu) -------------------------------------------
+int check_device(int* sm_count);   // W8_OK if the current device is sm_100; fills SM count
+
+// ---- quantizers (w8_quant.cu) --------------------------------------------------------
+int launch_quant_rows(int qfmt, const void* x, int M, int K, int ldx, void* q, float* scale, cudaStream_t s);
+int launch_quant_group128(const void* x, int M, int K, int ldx, void* q, float* scale, int ue8m0, cudaStream_t s);
+int launch_quant_weight_block(const void* w, int N, int K, void* q, float* scale, int ue8m0, cudaStream_t s);
+int launch_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, int ldx, void* q, float* scale,
+                         cudaStream_t s);
+int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float* scale, cudaStream_t s);
+
+constexpr int kRowMaxK = 32768;   // longest row the register-resident row kernels accept
+
+// ---- GEMM (w8_gemm.cu) -------------------------------------------------------------------
+enum : int { kTileBN16 = 0, kTileBN32, kTileBN64, kTileBN128, kTileBN256, kNumTiles };
+
+struct GemmPlan {
+    int fmt;          // W8_FMT_*
+    int M, N, K;
+    int swap;         // 1: Swap-AB (MMA M slot over N)
+    int bn;           // narrow tile side (16..256)
+    int split;        // split_k (power of two) when !stream
+    int stream;       // balanced partition over the SMs
+    int stages;
+    int pdl;
+    // derived
+    int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
+    long long units;
+    int G;
+    int align_tiles;
+    size_t ws_counters;   // bytes of the counter area (0 if no partials)
+    size_t ws_bytes;      // total workspace bytes
+    size_t smem_bytes;
+};
+
+int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);
+int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
+                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s);
+int gemm_device_status(int clear);
+
+// ---- per-shape variant table (w8_api.cu) ---------------------------------------------
+int table_lookup(int fmt, int N, int K, int M);   // explicit variant or 0 when absent
+
+}  // namespace w8

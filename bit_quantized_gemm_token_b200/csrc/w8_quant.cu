@@ -1,0 +1,465 @@
+// w8_quant.cu -- activation quantizers and the fused rms_norm / silu_and_mul producers.
+//
+// Definitions (the pages name these kernels in "PyTorch integra Helion en vLLM para
+// acelerar inferencia FP8", section "Kernels Helion implementados": dynamic_per_token_
+// scaled_fp8_quant, per_token_group_fp8_quant, rms_norm_dynamic_per_token_quant,
+// silu_and_mul_dynamic_per_token_quant; the fusions are the two pairs of section
+// "Patron de fusion del forward pass"):
+//   s = amax / Q (fp32 division; Q = 448 e4m3, 127 int8; s = 1 for an all-zero row),
+//   q = e4m3_rn_satfinite(x / s)  or  clamp(rint(x / s), -127, 127),
+//   UE8M0 scales: the smallest power of two >= amax/448, exponent in [-127, 127].
+// Every division is the IEEE one (__fdiv_rn), never x * (1/s), and no arithmetic is
+// left to compiler contraction (__fmul_rn / __fadd_rn / __fmaf_rn spell out each
+// rounding), so the codes are a deterministic function of the inputs.
+//
+// Layout of the work: the row kernels give one CTA per row and keep the row in
+// registers (16-byte vector loads, CPT chunks of 8 bf16 per thread); reductions are
+// warp shuffles plus one shared-memory stage.  The group kernel gives a half-warp per
+// 128-element group.  All kernels wait on the previous grid (programmatic dependent
+// launch) before reading and release their dependents right after.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "w8_internal.h"
+#include "w8_ptx.cuh"
+
+namespace w8 {
+namespace {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kInt8Max = 127.0f;
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8])
+{
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p)
+{
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Two fp32 -> two e4m3 codes (round to nearest even, saturating); element `lo` in the
+// low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t int8_code(float v)
+{
+    int r = __float2int_rn(v);   // ties to even; NaN -> 0
+    r = max(-127, min(127, r));
+    return static_cast<uint32_t>(r) & 0xFFu;
+}
+
+// 8 values / s -> 8 codes packed little-endian into a uint2.
+template <int QFMT>
+__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s)
+{
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(f[i], s);
+    uint2 r;
+    if (QFMT == W8_Q_FP8) {
+        r.x = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
+        r.y = e4m3x2(v[4], v[5]) | (e4m3x2(v[6], v[7]) << 16);
+    } else {
+        r.x = int8_code(v[0]) | (int8_code(v[1]) << 8) | (int8_code(v[2]) << 16) | (int8_code(v[3]) << 24);
+        r.y = int8_code(v[4]) | (int8_code(v[5]) << 8) | (int8_code(v[6]) << 16) | (int8_code(v[7]) << 24);
+    }
+    return r;
+}
+
+__device__ __forceinline__ float scale_from_amax(float amax, float qmax, bool ue8m0)
+{
+    if (!(amax > 0.0f)) return 1.0f;
+    float r = __fdiv_rn(amax, qmax);
+    if (!ue8m0) return r;
+    int e;
+    float f = frexpf(r, &e);          // r = f * 2^e exactly, f in [0.5, 1)
+    int p = (f == 0.5f) ? e - 1 : e;  // smallest power of two >= r
+    p = max(-127, min(127, p));
+    return ldexpf(1.0f, p);
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// Max over the CTA; every thread receives the result.  `red` holds 32 floats.
+__device__ __forceinline__ float block_max(float v, float* red)
+{
+    v = warp_max(v);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float r = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0f;
+    r = warp_max(r);
+    __syncthreads();
+    return r;
+}
+
+// Sum over the CTA in fp64 with a fixed reduction tree; every thread gets the result.
+__device__ __forceinline__ double block_sum_f64(double v, double* red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+    __syncthreads();
+    return r;
+}
+
+// exp(x) in fp32 by Cody & Waite's method: x = n ln2 + r with n = rint(x log2 e) and
+// ln2 split into a short leading part and a remainder, exp(r) by its Taylor series to
+// degree 7 (Horner, fused multiply-adds), and the exact scaling by 2^n as two
+// power-of-two factors that stay normal.  Each step is an explicitly rounded fp32 op,
+// so the result is fully specified (worst error about 1 ulp against exp).
+__device__ __forceinline__ float exp_cw(float x)
+{
+    if (x != x) return x;
+    if (x > 100.0f) return __int_as_float(0x7F800000);
+    if (x < -150.0f) return 0.0f;
+    const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));   // log2(e)
+    float r = __fmaf_rn(-n, 0x1.62e400p-1f, x);             // ln 2, leading bits
+    r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);                  // ln 2, remainder
+    float p = 0x1.a01a02p-13f;                              // 1/7!
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                   // 1/6!
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);                    // 1/5!
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);                    // 1/4!
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);                    // 1/3!
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    const int ni = static_cast<int>(n);
+    const int n1 = ni / 2, n2 = ni - n1;
+    return __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
+}
+
+// ------------------------------------------------------------------- per-token rows
+template <int QFMT, int CPT>
+__global__ void __launch_bounds__(1024) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int K, int ldx,
+                                                          uint8_t* __restrict__ q, float* __restrict__ scale)
+{
+    __shared__ float red[32];
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int m = blockIdx.x;
+    const int chunks = K >> 3;
+    const __nv_bfloat16* xr = x + (size_t)m * ldx;
+    uint4 raw[CPT];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            raw[c] = ld_nc_v4(xr + (size_t)idx * 8);
+            float f[8];
+            unpack_bf16x8(raw[c], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        }
+    }
+    amax = block_max(amax, red);
+    const float s = scale_from_amax(amax, QFMT == W8_Q_FP8 ? kE4M3Max : kInt8Max, false);
+    if (threadIdx.x == 0) scale[m] = s;
+    uint8_t* qr = q + (size_t)m * K;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            float f[8];
+            unpack_bf16x8(raw[c], f);
+            *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<QFMT>(f, s);
+        }
+    }
+}
+
+// ------------------------------------------------------------------- 1x128 groups
+// A half-warp (16 lanes x 8 elements) per group; scale[m * (K/128) + g].
+__global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
+                                                             int ldx, uint8_t* __restrict__ q,
+                                                             float* __restrict__ scale, int ue8m0)
+{
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int gpr = K >> 7;
+    const long long total = (long long)M * gpr;
+    const long long gid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
+    const int l16 = threadIdx.x & 15;
+    const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
+    if (gid >= total) return;   // whole half-warps leave together
+    const int m = (int)(gid / gpr), g = (int)(gid % gpr);
+    const uint4 raw = ld_nc_v4(x + (size_t)m * ldx + (size_t)g * 128 + l16 * 8);
+    float f[8];
+    unpack_bf16x8(raw, f);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
+    const float s = scale_from_amax(amax, kE4M3Max, ue8m0 != 0);
+    if (l16 == 0) scale[(size_t)m * gpr + g] = s;
+    *reinterpret_cast<uint2*>(q + (size_t)m * K + (size_t)g * 128 + l16 * 8) = encode8<W8_Q_FP8>(f, s);
+}
+
+// ------------------------------------------------------------------- 128x128 weight blocks
+__global__ void __launch_bounds__(256) quant_weight_block_kernel(const __nv_bfloat16* __restrict__ w, int N, int K,
+                                                                 uint8_t* __restrict__ q, float* __restrict__ scale,
+                                                                 int ue8m0)
+{
+    __shared__ float red[32];
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int bk = blockIdx.x, bn = blockIdx.y;
+    const int nbk = gridDim.x;
+    const int rows = min(128, N - bn * 128), cols = min(128, K - bk * 128);
+    uint4 raw[8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = threadIdx.x + i * 256;   // 16 chunks of 8 per row
+        const int r = c >> 4, cc = (c & 15) * 8;
+        if (r < rows && cc < cols) {
+            raw[i] = ld_nc_v4(w + (size_t)(bn * 128 + r) * K + bk * 128 + cc);
+            float f[8];
+            unpack_bf16x8(raw[i], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        }
+    }
+    amax = block_max(amax, red);
+    const float s = scale_from_amax(amax, kE4M3Max, ue8m0 != 0);
+    if (threadIdx.x == 0) scale[(size_t)bn * nbk + bk] = s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int c = threadIdx.x + i * 256;
+        const int r = c >> 4, cc = (c & 15) * 8;
+        if (r < rows && cc < cols) {
+            float f[8];
+            unpack_bf16x8(raw[i], f);
+            *reinterpret_cast<uint2*>(q + (size_t)(bn * 128 + r) * K + bk * 128 + cc) = encode8<W8_Q_FP8>(f, s);
+        }
+    }
+}
+
+// ------------------------------------------------------------------- rms_norm + quant
+template <int CPT>
+__global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16* __restrict__ x,
+                                                             const __nv_bfloat16* __restrict__ gamma, float eps,
+                                                             int H, int ldx, uint8_t* __restrict__ q,
+                                                             float* __restrict__ scale)
+{
+    __shared__ double redd[32];
+    __shared__ float red[32];
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int m = blockIdx.x;
+    const int chunks = H >> 3;
+    const __nv_bfloat16* xr = x + (size_t)m * ldx;
+    uint4 raw[CPT];
+    double ss = 0.0;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            raw[c] = ld_nc_v4(xr + (size_t)idx * 8);
+            float f[8];
+            unpack_bf16x8(raw[c], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const double d = (double)f[i];
+                ss = __fma_rn(d, d, ss);   // the square of a bf16 value is exact in fp64
+            }
+        }
+    }
+    ss = block_sum_f64(ss, redd);
+    const float mean = __fdiv_rn(__double2float_rn(ss), (float)H);
+    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+    // y = (x * r) * gamma, recomputed in the second pass rather than kept
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            float f[8], g[8];
+            unpack_bf16x8(raw[c], f);
+            unpack_bf16x8(ld_nc_v4(gamma + (size_t)idx * 8), g);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(f[i], r), g[i])));
+        }
+    }
+    amax = block_max(amax, red);
+    const float s = scale_from_amax(amax, kE4M3Max, false);
+    if (threadIdx.x == 0) scale[m] = s;
+    uint8_t* qr = q + (size_t)m * H;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            float f[8], g[8], y[8];
+            unpack_bf16x8(raw[c], f);
+            unpack_bf16x8(ld_nc_v4(gamma + (size_t)idx * 8), g);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(f[i], r), g[i]);
+            *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<W8_Q_FP8>(y, s);
+        }
+    }
+}
+
+// ------------------------------------------------------------------- silu_and_mul + quant
+template <int CPT>
+__global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat16* __restrict__ xgu, int I, int ld,
+                                                              uint8_t* __restrict__ q, float* __restrict__ scale)
+{
+    __shared__ float red[32];
+    ptx::grid_dep_wait();
+    ptx::grid_dep_launch();
+    const int m = blockIdx.x;
+    const int chunks = I >> 3;
+    const __nv_bfloat16* gr = xgu + (size_t)m * ld;
+    const __nv_bfloat16* ur = gr + I;
+    float h[CPT][8];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) {
+            float g[8], u[8];
+            unpack_bf16x8(ld_nc_v4(gr + (size_t)idx * 8), g);
+            unpack_bf16x8(ld_nc_v4(ur + (size_t)idx * 8), u);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float den = __fadd_rn(1.0f, exp_cw(-g[i]));
+                h[c][i] = __fmul_rn(__fdiv_rn(g[i], den), u[i]);
+                amax = fmaxf(amax, fabsf(h[c][i]));
+            }
+        }
+    }
+    amax = block_max(amax, red);
+    const float s = scale_from_amax(amax, kE4M3Max, false);
+    if (threadIdx.x == 0) scale[m] = s;
+    uint8_t* qr = q + (size_t)m * I;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<W8_Q_FP8>(h[c], s);
+    }
+}
+
+// Threads per row and chunks per thread for a row of `chunks` 16-byte chunks: the
+// fewest chunks per thread (1, 2 or 4) that fits in 1024 threads.
+inline bool row_shape(int chunks, int* threads, int* cpt)
+{
+    for (int c : {1, 2, 4}) {
+        const int t = (chunks + c - 1) / c;
+        if (t <= 1024) {
+            *cpt = c;
+            *threads = ((t + 31) / 32) * 32;
+            if (*threads < 64) *threads = 64;
+            return true;
+        }
+    }
+    return false;
+}
+
+cudaError_t launch(const void* fn, dim3 grid, dim3 block, void** args, cudaStream_t s)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? W8_OK : W8_ERR_CUDA; }
+
+}  // namespace
+
+int launch_quant_rows(int qfmt, const void* x, int M, int K, int ldx, void* q, float* scale, cudaStream_t s)
+{
+    int threads, cpt;
+    if (!row_shape(K / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
+    uint8_t* qp = static_cast<uint8_t*>(q);
+    void* args[] = {(void*)&xp, (void*)&K, (void*)&ldx, (void*)&qp, (void*)&scale};
+    const void* fn = nullptr;
+    if (qfmt == W8_Q_FP8)
+        fn = cpt == 1 ? (const void*)quant_rows_kernel<W8_Q_FP8, 1>
+                      : cpt == 2 ? (const void*)quant_rows_kernel<W8_Q_FP8, 2> : (const void*)quant_rows_kernel<W8_Q_FP8, 4>;
+    else
+        fn = cpt == 1 ? (const void*)quant_rows_kernel<W8_Q_INT8, 1>
+                      : cpt == 2 ? (const void*)quant_rows_kernel<W8_Q_INT8, 2>
+                                 : (const void*)quant_rows_kernel<W8_Q_INT8, 4>;
+    return status_of(launch(fn, dim3(M), dim3(threads), args, s));
+}
+
+int launch_quant_group128(const void* x, int M, int K, int ldx, void* q, float* scale, int ue8m0, cudaStream_t s)
+{
+    const long long threads = (long long)M * (K / 128) * 16;
+    const long long blocks = (threads + 255) / 256;
+    if (blocks > 0x7FFFFFFF) return W8_ERR_UNSUPPORTED;
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
+    uint8_t* qp = static_cast<uint8_t*>(q);
+    void* args[] = {(void*)&xp, (void*)&M, (void*)&K, (void*)&ldx, (void*)&qp, (void*)&scale, (void*)&ue8m0};
+    return status_of(launch((const void*)quant_group128_kernel, dim3((unsigned)blocks), dim3(256), args, s));
+}
+
+int launch_quant_weight_block(const void* w, int N, int K, void* q, float* scale, int ue8m0, cudaStream_t s)
+{
+    const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(w);
+    uint8_t* qp = static_cast<uint8_t*>(q);
+    void* args[] = {(void*)&wp, (void*)&N, (void*)&K, (void*)&qp, (void*)&scale, (void*)&ue8m0};
+    dim3 grid((K + 127) / 128, (N + 127) / 128);
+    if (grid.y > 65535) return W8_ERR_UNSUPPORTED;
+    return status_of(launch((const void*)quant_weight_block_kernel, grid, dim3(256), args, s));
+}
+
+int launch_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, int ldx, void* q, float* scale,
+                         cudaStream_t s)
+{
+    int threads, cpt;
+    if (!row_shape(H / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(gamma);
+    uint8_t* qp = static_cast<uint8_t*>(q);
+    void* args[] = {(void*)&xp, (void*)&gp, (void*)&eps, (void*)&H, (void*)&ldx, (void*)&qp, (void*)&scale};
+    const void* fn = cpt == 1 ? (const void*)rmsnorm_quant_kernel<1>
+                              : cpt == 2 ? (const void*)rmsnorm_quant_kernel<2> : (const void*)rmsnorm_quant_kernel<4>;
+    return status_of(launch(fn, dim3(M), dim3(threads), args, s));
+}
+
+int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float* scale, cudaStream_t s)
+{
+    int threads, cpt;
+    if (!row_shape(I / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
+    const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(xgu);
+    uint8_t* qp = static_cast<uint8_t*>(q);
+    void* args[] = {(void*)&xp, (void*)&I, (void*)&ld, (void*)&qp, (void*)&scale};
+    const void* fn = cpt == 1 ? (const void*)silu_mul_quant_kernel<1>
+                              : cpt == 2 ? (const void*)silu_mul_quant_kernel<2> : (const void*)silu_mul_quant_kernel<4>;
+    return status_of(launch(fn, dim3(M), dim3(threads), args, s));
+}
+
+}  // namespace w8

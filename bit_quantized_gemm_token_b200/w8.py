@@ -1,0 +1,285 @@
+"""Python binding of libw8 (include/w8.h): the same entry points, argument marshalling
+only.  Every step of the layer runs in the library's CUDA kernels; there is no CPU or
+PyTorch-op fallback, and using any entry point without the built library raises.
+
+Tensors are torch CUDA tensors.  Outputs may be passed in (for graph capture) or are
+allocated here with torch (allocation is plumbing, not compute).  Calls are enqueued
+on torch's current stream unless `stream` is given.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libw8.so")
+
+# status codes
+W8_OK = 0
+W8_ERR_INVALID_ARG = -1
+W8_ERR_UNSUPPORTED = -2
+W8_ERR_ALIGNMENT = -3
+W8_ERR_WORKSPACE = -4
+W8_ERR_CUDA = -5
+W8_ERR_DEVICE_TIMEOUT = -6
+W8_ERR_NO_DEVICE = -7
+W8_ERR_IO = -8
+
+W8_Q_FP8, W8_Q_INT8 = 0, 1
+W8_FMT_FP8_DYN, W8_FMT_INT8, W8_FMT_BLOCK_FP8, W8_FMT_BLOCK_FP8_UE8M0 = 0, 1, 2, 3
+
+W8_VARIANT_AUTO = 0
+W8_V_EXPLICIT = 1 << 0
+W8_V_SWAP_AB = 1 << 1
+W8_V_STREAM = 1 << 2
+W8_V_SPLIT_SHIFT = 4
+W8_V_TILE_SHIFT = 8
+W8_V_STAGES_SHIFT = 12
+W8_V_PDL = 1 << 16
+TILE_BN = {16: 0, 32: 1, 64: 2, 128: 3, 256: 4}
+
+
+def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stages: int = 0, pdl: bool = False) -> int:
+    """Explicit variant word (the W8_VARIANT macro plus stages / PDL bits)."""
+    lg = int(split).bit_length() - 1
+    if split < 1 or (1 << lg) != split:
+        raise ValueError("split must be a power of two")
+    v = W8_V_EXPLICIT | (W8_V_SWAP_AB if swap else 0) | (W8_V_STREAM if stream else 0)
+    v |= (lg & 0xF) << W8_V_SPLIT_SHIFT
+    v |= (TILE_BN[bn] & 0xF) << W8_V_TILE_SHIFT
+    v |= (stages & 0xF) << W8_V_STAGES_SHIFT
+    if pdl:
+        v |= W8_V_PDL
+    return v
+
+
+def describe(v: int) -> dict:
+    inv = {b: k for k, b in TILE_BN.items()}
+    return {"swap_ab": bool(v & W8_V_SWAP_AB), "stream": bool(v & W8_V_STREAM),
+            "split_k": 1 << ((v >> W8_V_SPLIT_SHIFT) & 0xF), "bn": inv.get((v >> W8_V_TILE_SHIFT) & 0xF),
+            "stages": (v >> W8_V_STAGES_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL)}
+
+
+class W8Error(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__("%s failed: %s (%d)" % (fn, status_string(code), code))
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libw8.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libw8.so is not built: run `python -m bit_quantized_gemm_token_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.w8_quant_per_token.argtypes = [I, P, I, I, I, P, P, I, I, P]
+    L.w8_quant_weight_block.argtypes = [P, I, I, P, P, I, P]
+    L.w8_rmsnorm_quant.argtypes = [P, P, F, I, I, I, P, P, P]
+    L.w8_silu_mul_quant.argtypes = [P, I, I, I, P, P, P]
+    L.w8_gemm.argtypes = [I, P, P, P, P, P, I, I, I, I, P, S, P]
+    L.w8_gemm_workspace_size.argtypes = [I, I, I, I, I]
+    L.w8_gemm_workspace_size.restype = S
+    L.w8_gemm_resolve_variant.argtypes = [I, I, I, I, I]
+    L.w8_gemm_i32_debug.argtypes = [P, P, P, I, I, I, I, P, S, P]
+    L.w8_load_table.argtypes = [ctypes.c_char_p]
+    L.w8_clear_table.argtypes = []
+    L.w8_clear_table.restype = None
+    L.w8_device_status.argtypes = [I]
+    L.w8_status_string.argtypes = [I]
+    L.w8_status_string.restype = ctypes.c_char_p
+    L.w8_version.argtypes = []
+    for fn in ("w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant", "w8_gemm",
+               "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
+        getattr(L, fn).restype = I
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().w8_status_string(int(code)).decode()
+
+
+def _check(fn, rc):
+    if rc != W8_OK:
+        raise W8Error(fn, rc)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name):
+    if t.dtype != dtype or not t.is_cuda:
+        raise TypeError("%s must be a CUDA %s tensor (got %s on %s)" % (name, dtype, t.dtype, t.device))
+
+
+# ---------------------------------------------------------------------------- quantizers
+
+def w8_quant_per_token(x, qfmt=W8_Q_FP8, group=0, ue8m0=False, q=None, scale=None, stream=None):
+    """bf16 x[M, K] (row stride x.stride(0)) -> (codes[M, K], scales [M] or [M, K/group])."""
+    _need(x, torch.bfloat16, "x")
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    M, K = x.shape
+    qdt = torch.float8_e4m3fn if qfmt == W8_Q_FP8 else torch.int8
+    if q is None:
+        q = torch.empty((M, K), dtype=qdt, device=x.device)
+    if scale is None:
+        scale = torch.empty((M,) if group == 0 else (M, K // group), dtype=torch.float32, device=x.device)
+    rc = lib().w8_quant_per_token(qfmt, _ptr(x), M, K, x.stride(0), _ptr(q), _ptr(scale), group, int(bool(ue8m0)),
+                                  _stream(stream))
+    _check("w8_quant_per_token", rc)
+    return q, scale
+
+
+def w8_quant_weight_block(w, ue8m0=False, q=None, scale=None, stream=None):
+    """bf16 W[N, K] -> (e4m3 codes [N, K], scales [ceil(N/128), ceil(K/128)])."""
+    _need(w, torch.bfloat16, "w")
+    N, K = w.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    if scale is None:
+        scale = torch.empty(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=w.device)
+    rc = lib().w8_quant_weight_block(_ptr(w.contiguous()), N, K, _ptr(q), _ptr(scale), int(bool(ue8m0)),
+                                     _stream(stream))
+    _check("w8_quant_weight_block", rc)
+    return q, scale
+
+
+def w8_rmsnorm_quant(x, gamma, eps=1e-6, q=None, scale=None, stream=None):
+    _need(x, torch.bfloat16, "x")
+    _need(gamma, torch.bfloat16, "gamma")
+    M, H = x.shape
+    if q is None:
+        q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    rc = lib().w8_rmsnorm_quant(_ptr(x), _ptr(gamma), float(eps), M, H, x.stride(0), _ptr(q), _ptr(scale),
+                                _stream(stream))
+    _check("w8_rmsnorm_quant", rc)
+    return q, scale
+
+
+def w8_silu_mul_quant(gate_up, q=None, scale=None, stream=None):
+    """bf16 gate_up[M, 2I] (gate first) -> (e4m3 codes of silu(gate)*up [M, I], scales [M])."""
+    _need(gate_up, torch.bfloat16, "gate_up")
+    M, I2 = gate_up.shape
+    I = I2 // 2
+    if q is None:
+        q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    if scale is None:
+        scale = torch.empty((M,), dtype=torch.float32, device=gate_up.device)
+    rc = lib().w8_silu_mul_quant(_ptr(gate_up), M, I, gate_up.stride(0), _ptr(q), _ptr(scale), _stream(stream))
+    _check("w8_silu_mul_quant", rc)
+    return q, scale
+
+
+# ---------------------------------------------------------------------------- GEMM
+
+def w8_gemm_workspace_size(fmt, M, N, K, variant=W8_VARIANT_AUTO):
+    n = lib().w8_gemm_workspace_size(fmt, M, N, K, variant)
+    if n == ctypes.c_size_t(-1).value:
+        raise W8Error("w8_gemm_workspace_size", W8_ERR_INVALID_ARG)
+    return n
+
+
+def w8_gemm_resolve_variant(fmt, M, N, K, variant=W8_VARIANT_AUTO):
+    v = lib().w8_gemm_resolve_variant(fmt, M, N, K, variant)
+    if v < 0:
+        raise W8Error("w8_gemm_resolve_variant", v)
+    return v
+
+
+class Workspace:
+    """A zero-initialised device scratch buffer for w8_gemm, grown on demand (growth
+    re-zeroes).  Calls sharing one workspace must be ordered on one stream."""
+
+    def __init__(self, device=None, nbytes=0):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+        if nbytes:
+            self.reserve(nbytes)
+
+    def reserve(self, nbytes):
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+    def args(self, nbytes):
+        if nbytes == 0:
+            return None, 0
+        b = self.reserve(nbytes)
+        return ctypes.c_void_p(b.data_ptr()), b.numel()
+
+
+_default_ws = {}
+
+
+def _workspace(ws, device, nbytes):
+    if ws is None:
+        ws = _default_ws.setdefault(device, Workspace(device))
+    return ws.args(nbytes)
+
+
+def w8_gemm(fmt, A_q, A_scale, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
+    """out[M, N] (bf16) = scaled A_q . W_q^T in format `fmt` (W8_FMT_*)."""
+    M, K = A_q.shape
+    N = W_q.shape[0]
+    if W_q.shape[1] != K:
+        raise ValueError("K mismatch")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
+    _need(out, torch.bfloat16, "out")
+    nbytes = w8_gemm_workspace_size(fmt, M, N, K, variant)
+    wp, wn = _workspace(workspace, A_q.device, nbytes)
+    rc = lib().w8_gemm(fmt, _ptr(A_q), _ptr(A_scale), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp, wn,
+                       _stream(stream))
+    _check("w8_gemm", rc)
+    return out
+
+
+def w8_gemm_i32_debug(A_q, W_q, acc=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
+    """Raw int32 accumulators acc[M, N] = sum_k A_q W_q (INT8 path, no scales)."""
+    M, K = A_q.shape
+    N = W_q.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=A_q.device)
+    nbytes = w8_gemm_workspace_size(W8_FMT_INT8, M, N, K, variant)
+    wp, wn = _workspace(workspace, A_q.device, nbytes)
+    rc = lib().w8_gemm_i32_debug(_ptr(A_q), _ptr(W_q), _ptr(acc), M, N, K, variant, wp, wn, _stream(stream))
+    _check("w8_gemm_i32_debug", rc)
+    return acc
+
+
+def w8_load_table(path):
+    n = lib().w8_load_table(os.fsencode(path))
+    if n < 0:
+        raise W8Error("w8_load_table", n)
+    return n
+
+
+def w8_clear_table():
+    lib().w8_clear_table()
+
+
+def w8_device_status(clear=True):
+    return lib().w8_device_status(int(bool(clear)))
+
+
+def w8_status_string(code):
+    return status_string(code)
+
+
+def w8_version():
+    return lib().w8_version()

@@ -1,0 +1,212 @@
+/*
+ * w8.h -- C ABI of libw8, the B200 (sm_100a) 8-bit quantized linear layer.
+ *
+ * The layer is a dynamic activation quantizer (or a fused rms_norm / silu_and_mul
+ * producer) feeding one scaled GEMM that covers the Standard, Split-K and Swap-AB
+ * variants in three 8-bit formats: FP8-dynamic, W8A8-INT8 and Block-FP8.  Sources
+ * (web pages; no formulas are printed there, so each entry point states the
+ * definition it computes):
+ *   [FP8] "PyTorch integra Helion en vLLM para acelerar inferencia FP8"
+ *         (noticias.mechatronicstore.cl) -- sections "Patron de fusion del forward
+ *         pass" (rms_norm + fp8_quant, silu_and_mul + fp8_quant, scaled_mm as the
+ *         linear op) and "Kernels Helion implementados" (the kernel list);
+ *   [LIN] "Helion DSL added to vLLM to autotune linear inference backends"
+ *         (signaltitans.com) -- "Unified GEMM Architecture" (one GEMM, Split-K and
+ *         Swap-AB as parameters, FP8 Dynamic / W8A8 INT8 / Block FP8) and "Hybrid
+ *         Dispatch and Autotuning" (small token counts under CUDA-graph replay);
+ *   [IT]  "Helion nel backend vLLM: un solo GEMM, tuning per forma e guadagni fino
+ *         al 10%" (ai-radar.it) -- paragraphs 2-4 (Split-K, Swap-AB as (B^T A^T)^T,
+ *         split_k a power of two up to 256, per-shape configs).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are DEVICE memory owned by the caller; the library never allocates
+ *     device memory on these paths and never synchronises: every call only enqueues
+ *     work on `stream` (NULL = the legacy default stream) and returns.
+ *   - Layouts are row-major.  M = tokens, K = in-features, N = out-features.
+ *     Activations x are bf16 [M, K] with row stride ldx (elements).  Codes are one byte
+ *     each: e4m3 ("fn": max 448, no inf) or int8 in [-127, 127].  Weights are
+ *     W[N, K] (K contiguous; the nn.Linear [out, in] layout).  GEMM output is bf16
+ *     [M, N].  Scales are fp32.
+ *   - Every call returns W8_OK (0) or a negative W8_ERR_* code; on an error nothing
+ *     was enqueued.  No call aborts the process or traps on the device.
+ *   - Quantization: s = amax / Q with Q = 448 (e4m3) or 127 (int8), an IEEE fp32
+ *     division; codes = RNE(x / s) (true division), e4m3 saturating to +-448, int8
+ *     clamped to [-127, 127].  An all-zero row or group gets s = 1 (codes 0).
+ *     UE8M0 scales are s = 2^ceil(log2(amax/448)) (fp32 quotient), exponent clamped to
+ *     [-127, 127]; they are still passed as fp32 values.
+ *   - Input values are expected to be finite.
+ */
+#ifndef W8_H
+#define W8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
+
+#if defined(__GNUC__)
+#define W8_API __attribute__((visibility("default")))
+#else
+#define W8_API
+#endif
+
+/* ---- status codes ---------------------------------------------------------- */
+#define W8_OK 0
+#define W8_ERR_INVALID_ARG (-1)     /* null pointer, non-positive size, bad enum     */
+#define W8_ERR_UNSUPPORTED (-2)     /* format / variant / size not available          */
+#define W8_ERR_ALIGNMENT (-3)       /* pointer or stride not aligned as required      */
+#define W8_ERR_WORKSPACE (-4)       /* workspace missing or smaller than required     */
+#define W8_ERR_CUDA (-5)            /* a CUDA runtime call (e.g. the launch) failed   */
+#define W8_ERR_DEVICE_TIMEOUT (-6)  /* a bounded device-side wait gave up             */
+#define W8_ERR_NO_DEVICE (-7)       /* current device is not an sm_100 (B200) part    */
+#define W8_ERR_IO (-8)              /* table file missing or malformed                */
+
+/* ---- activation quantizer formats ------------------------------------------ */
+#define W8_Q_FP8 0
+#define W8_Q_INT8 1
+
+/* ---- GEMM formats -------------------------------------------------------------- */
+#define W8_FMT_FP8_DYN 0          /* per-token sA[M] x per-channel sW[N]                  */
+#define W8_FMT_INT8 1             /* same scales, int8 x int8 -> int32 accumulation       */
+#define W8_FMT_BLOCK_FP8 2        /* sA[M, K/128] (1x128 groups), sW[N/128, K/128] blocks */
+#define W8_FMT_BLOCK_FP8_UE8M0 3  /* as BLOCK_FP8, every scale an exact power of two      */
+
+/* ---- GEMM variant word -----------------------------------------------------------
+ * 0 (W8_VARIANT_AUTO) lets the library choose from its per-shape table (loaded with
+ * w8_load_table) or, when the shape is not in it, from a built-in rule.  An explicit
+ * variant sets W8_V_EXPLICIT plus:
+ *   W8_V_SWAP_AB  compute out^T = W . Aq^T: the 128-row MMA slot runs over N and the
+ *                 narrow slot over tokens (the Swap-AB variant, for small M);
+ *                 otherwise the 128-row slot runs over tokens (Standard).
+ *   split         log2 of split_k in bits 4..7 (split_k = 1..256, a power of two,
+ *                 <= ceil(K/128)): every output tile's K range is cut into split_k
+ *                 chunks, one CTA each, and the fp32 (int32 for INT8) partials are
+ *                 added in a fixed order (Split-K).  split = 0 without W8_V_STREAM is
+ *                 the Standard full-K tile loop.
+ *   W8_V_STREAM   balanced partition: the (tile, 128-column K block) units are dealt
+ *                 out evenly to one CTA per SM, so a tile's K range may be split across
+ *                 neighbouring CTAs (a Split-K whose chunk boundaries follow the SM
+ *                 count); split bits are ignored.
+ *   tile          bits 8..11, the narrow tile side BN: 0:16 1:32 2:64 3:128 4:256.
+ *   stages        bits 12..15, shared-memory pipeline depth (0 = default).
+ *   W8_V_PDL      launch with programmatic dependent launch: the kernel starts while
+ *                 the previous kernel on the stream finishes and streams weight tiles
+ *                 before waiting for it.  Only legal when W_q and the scales of W were
+ *                 NOT written by the kernel launched immediately before this one.
+ */
+#define W8_VARIANT_AUTO 0
+#define W8_V_EXPLICIT (1 << 0)
+#define W8_V_SWAP_AB (1 << 1)
+#define W8_V_STREAM (1 << 2)
+#define W8_V_SPLIT_SHIFT 4
+#define W8_V_TILE_SHIFT 8
+#define W8_V_STAGES_SHIFT 12
+#define W8_V_PDL (1 << 16)
+#define W8_VARIANT(swap, log2_split, tile, stream)                                            \
+    (W8_V_EXPLICIT | ((swap) ? W8_V_SWAP_AB : 0) | ((stream) ? W8_V_STREAM : 0) |            \
+     (((log2_split) & 0xF) << W8_V_SPLIT_SHIFT) | (((tile) & 0xF) << W8_V_TILE_SHIFT))
+
+/* ---- entry points ---------------------------------------------------------------- */
+
+/* Dynamic per-token (group == 0) or per-token-group (group == 128) quantization.
+ * [FP8] "Kernels Helion implementados": dynamic_per_token_scaled_fp8_quant and
+ * per_token_group_fp8_quant; the int8 form is the W8A8 INT8 activation side of [LIN]
+ * "Unified GEMM Architecture".
+ *   qfmt   W8_Q_FP8 or W8_Q_INT8 (group > 0 and ue8m0 need W8_Q_FP8)
+ *   x      bf16 [M, K], row stride ldx >= K; 16-byte aligned, ldx % 8 == 0, K % 8 == 0
+ *   q      codes [M, K], row stride K (bytes); 8-byte aligned
+ *   scale  fp32 [M] (group == 0) or [M, K/group] (K % group == 0)
+ *   ue8m0  nonzero: power-of-two scales (group mode only)
+ * Limits: K <= 32768 for group == 0.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA.
+ * Also the offline per-output-channel weight quantizer: pass W[N, K] as x (M = N). */
+W8_API int w8_quant_per_token(int qfmt, const void* x, int M, int K, int ldx, void* q, float* scale, int group,
+                       int ue8m0, w8_stream_t stream);
+
+/* Block-FP8 weight quantization (offline weight preparation for W8_FMT_BLOCK_FP8*):
+ * one scale per 128x128 block of W, s = amax(block)/448 (or its UE8M0 power of two),
+ * codes e4m3(w / s).  [FP8] "Kernels Helion implementados" (scaled_mm_blockwise
+ * consumes weights in this form).
+ *   w      bf16 [N, K] contiguous, 16-byte aligned, K % 8 == 0
+ *   q      e4m3 [N, K]; scale fp32 [ceil(N/128), ceil(K/128)] */
+W8_API int w8_quant_weight_block(const void* w, int N, int K, void* q, float* scale, int ue8m0, w8_stream_t stream);
+
+/* Fused rms_norm + dynamic per-token fp8 quant, one launch ([FP8] "Patron de fusion
+ * del forward pass": rms_norm + fp8_quant; "Kernels Helion implementados":
+ * rms_norm_dynamic_per_token_quant).  Per row:
+ *   ss = sum x^2 accumulated in fp64, rounded to fp32; r = 1/sqrt(ss/H + eps) (fp32,
+ *   correctly rounded steps); y = (x * r) * gamma in fp32 (never rounded to bf16);
+ *   then the per-token fp8 quantization of y.
+ *   x bf16 [M, H] (row stride ldx), gamma bf16 [H]; q e4m3 [M, H]; scale fp32 [M].
+ * Same alignment rules and limits as w8_quant_per_token (H in place of K). */
+W8_API int w8_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, int ldx, void* q, float* scale,
+                     w8_stream_t stream);
+
+/* Fused silu_and_mul + dynamic per-token fp8 quant, one launch ([FP8] "Kernels Helion
+ * implementados": silu_and_mul_dynamic_per_token_quant).  Row m of gate_up [M, 2I]
+ * (row stride ld) holds the gate in columns [0, I) and the up projection in [I, 2I);
+ * h = (g / (1 + exp(-g))) * u in fp32 with the library's own correctly specified exp
+ * (Cody-Waite reduction, degree-7 polynomial), then per-token fp8 quant of h.
+ *   q e4m3 [M, I]; scale fp32 [M].  I % 8 == 0, ld % 8 == 0, 16-byte aligned. */
+W8_API int w8_silu_mul_quant(const void* gate_up, int M, int I, int ld, void* q, float* scale, w8_stream_t stream);
+
+/* Scaled 8-bit GEMM, out = A . W^T with the format's scales, as ONE kernel family whose
+ * Standard, Split-K and Swap-AB forms are chosen by `variant` ([LIN] "Unified GEMM
+ * Architecture"; [IT] paragraphs 2-3; [FP8] "Kernels Helion implementados":
+ * scaled_mm, scaled_mm_blockwise):
+ *   FP8_DYN : out[m,n] = bf16( (sum_k a*w) * sA[m] * sW[n] ), fp32 accumulation
+ *   INT8    : out[m,n] = bf16( float(sum_k a*w as int32) * sA[m] * sW[n] )
+ *   BLOCK   : out[m,n] = bf16( sum_kb sA[m,kb] * sW[n/128,kb] * (sum_{k in kb} a*w) )
+ *   A_q      codes [M, K], row-major, 16-byte aligned; K % 16 == 0 (K % 128 for BLOCK)
+ *   A_scale  fp32 [M] or [M, K/128] (BLOCK)
+ *   W_q      codes [N, K], row-major, 16-byte aligned
+ *   W_scale  fp32 [N] or [ceil(N/128), K/128] (BLOCK)
+ *   out      bf16 [M, N], row-major
+ *   workspace/ws_bytes  scratch for split partials and tile counters, sized by
+ *            w8_gemm_workspace_size for the same (fmt, M, N, K, variant).  It must be
+ *            zero-filled once before its first use; every successful call leaves its
+ *            counter area zero again.  May be NULL when the size is 0.  Calls that
+ *            share a workspace must not overlap on the device.
+ * Accuracy: max|out - ref| <= 2^-7 max|ref| + 1e-3 against the fp64 definition.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, NO_DEVICE, CUDA. */
+W8_API int w8_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale, void* out,
+            int M, int N, int K, int variant, void* workspace, size_t ws_bytes, w8_stream_t stream);
+
+/* Bytes of workspace w8_gemm needs for this call (0 if none); (size_t)-1 if the
+ * arguments are invalid.  AUTO is resolved exactly as w8_gemm resolves it. */
+W8_API size_t w8_gemm_workspace_size(int fmt, int M, int N, int K, int variant);
+
+/* The explicit variant word AUTO resolves to for this shape (table, else built-in
+ * rule), or an explicit `variant` validated and returned unchanged; negative
+ * W8_ERR_* if illegal for the shape. */
+W8_API int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant);
+
+/* INT8 GEMM that writes the raw int32 accumulators acc[M, N] = sum_k a*w (no scales,
+ * no bf16), through the same kernels and variants as w8_gemm.  For bit-exact checks
+ * of the integer path. */
+W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int N, int K, int variant,
+                      void* workspace, size_t ws_bytes, w8_stream_t stream);
+
+/* Per-shape variant table (the output of the offline sweep).  Text, one entry per line:
+ *   <fmt> <N> <K> <m_max> <variant as 0x hex>
+ * '#' starts a comment.  AUTO picks the entry with the same (fmt, N, K) and the
+ * smallest m_max >= M.  Loading replaces the previous table.  Returns the number of
+ * entries, or W8_ERR_IO / W8_ERR_INVALID_ARG. */
+W8_API int w8_load_table(const char* path);
+W8_API void w8_clear_table(void);
+
+/* Device-side error word (set by a kernel whose bounded wait gave up): returns 0 or a
+ * W8_ERR_* code for the current device; clears it when `clear` is nonzero.  Reads
+ * device memory synchronously: call after the work in question has completed. */
+W8_API int w8_device_status(int clear);
+
+W8_API const char* w8_status_string(int status);
+W8_API int w8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* W8_H */

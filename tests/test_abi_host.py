@@ -1,0 +1,109 @@
+"""Host-only checks of the C ABI: the library builds and loads, exports every entry
+point include/w8.h declares, and rejects bad arguments with the documented status
+codes before touching a device.  No compute call runs here (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_gemm_token_b200 import build, w8
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return w8.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "w8.h")).read()
+    return re.findall(r"W8_API\s+[\w\s\*]+?\b(w8_\w+)\s*\(", src)
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(0, -9, -1):
+        s = w8.status_string(code)
+        assert s and s != "unknown status", code
+    assert w8.status_string(-99) == "unknown status"
+    assert w8.w8_version() >= 1
+
+
+NULL = None
+
+
+def test_bad_arguments_rejected_before_device(L):
+    # null pointers / sizes
+    assert L.w8_gemm(0, NULL, NULL, NULL, NULL, NULL, 1, 1, 16, 0, NULL, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    p16 = ctypes.c_void_p(1 << 20)           # aligned dummies: never dereferenced on these paths
+    podd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.w8_gemm(0, p16, p16, p16, p16, p16, 0, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    assert L.w8_gemm(0, podd, p16, p16, p16, p16, 1, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_ALIGNMENT
+    assert L.w8_quant_per_token(0, NULL, 1, 16, 16, p16, p16, 0, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    assert L.w8_quant_per_token(0, p16, 1, 12, 12, p16, p16, 0, 0, NULL) == w8.W8_ERR_ALIGNMENT
+    assert L.w8_quant_per_token(5, p16, 1, 16, 16, p16, p16, 0, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    assert L.w8_quant_per_token(1, p16, 1, 256, 256, p16, p16, 128, 0, NULL) == w8.W8_ERR_UNSUPPORTED
+    assert L.w8_quant_per_token(0, p16, 1, 256, 256, p16, p16, 64, 0, NULL) == w8.W8_ERR_UNSUPPORTED
+    assert L.w8_quant_per_token(0, p16, 1, 65536, 65536, p16, p16, 0, 0, NULL) == w8.W8_ERR_UNSUPPORTED
+    assert L.w8_rmsnorm_quant(p16, NULL, ctypes.c_float(1e-6), 1, 16, 16, p16, p16, NULL) == w8.W8_ERR_INVALID_ARG
+    assert L.w8_silu_mul_quant(p16, 1, 16, 16, p16, p16, NULL) == w8.W8_ERR_INVALID_ARG   # ld < 2I
+    assert L.w8_gemm_i32_debug(p16, p16, NULL, 1, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_INVALID_ARG
+
+
+def test_valid_call_without_device_reports_no_device(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    p16 = ctypes.c_void_p(1 << 20)
+    assert L.w8_quant_per_token(0, p16, 1, 16, 16, p16, p16, 0, 0, NULL) == w8.W8_ERR_NO_DEVICE
+    assert L.w8_gemm(0, p16, p16, p16, p16, p16, 1, 128, 128, 0, NULL, 0, NULL) == w8.W8_ERR_NO_DEVICE
+
+
+def test_variant_resolution_and_workspace(L):
+    # decode: Swap-AB with the narrow token tile, balanced partition
+    v = w8.w8_gemm_resolve_variant(0, 1, 4096, 4096)
+    d = w8.describe(v)
+    assert d["swap_ab"] and d["stream"] and d["bn"] == 16
+    assert w8.describe(w8.w8_gemm_resolve_variant(0, 32, 4096, 4096))["bn"] == 32
+    assert not w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["swap_ab"]
+    # explicit variants are validated
+    assert L.w8_gemm_resolve_variant(0, 8, 256, 1024, w8.variant(True, split=4, bn=16)) > 0
+    assert L.w8_gemm_resolve_variant(0, 8, 256, 256, w8.variant(True, split=4, bn=16)) == w8.W8_ERR_UNSUPPORTED  # 4 > 2 K blocks
+    assert L.w8_gemm_resolve_variant(2, 8, 256, 256, w8.variant(True, bn=128)) == w8.W8_ERR_UNSUPPORTED  # block needs BN <= 64
+    assert L.w8_gemm_resolve_variant(0, 8, 256, 200, 0) == w8.W8_ERR_ALIGNMENT          # K % 16
+    assert L.w8_gemm_resolve_variant(2, 8, 256, 144, 0) == w8.W8_ERR_ALIGNMENT          # block K % 128
+    # workspace: none for whole-tile partitions, some for split / balanced
+    assert w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=1, bn=16)) == 0
+    n = w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=4, bn=16))
+    tiles = 2
+    assert n == 256 + tiles * 4 * 2 * 16 * 128 * 4
+    assert w8.w8_gemm_workspace_size(0, 8, 4096, 4096, 0) > 0
+
+
+def test_table_parsing(L, tmp_path):
+    p = tmp_path / "t.txt"
+    v1 = w8.variant(True, split=2, bn=32)
+    v2 = w8.variant(False, split=1, bn=128)
+    p.write_text("# comment\n0 4096 4096 16 0x%x\n\n0 4096 4096 4096 0x%x  # prefill\n" % (v1, v2))
+    try:
+        assert w8.w8_load_table(str(p)) == 2
+        assert w8.w8_gemm_resolve_variant(0, 8, 4096, 4096) == v1
+        assert w8.w8_gemm_resolve_variant(0, 17, 4096, 4096) == v2
+        assert w8.describe(w8.w8_gemm_resolve_variant(0, 8, 4096, 6144))["stream"]   # not in table
+        bad = tmp_path / "bad.txt"
+        bad.write_text("0 4096 4096 16\n")
+        assert L.w8_load_table(os.fsencode(str(bad))) == w8.W8_ERR_IO
+        assert L.w8_load_table(b"/nonexistent/table.txt") == w8.W8_ERR_IO
+        assert w8.w8_gemm_resolve_variant(0, 8, 4096, 4096) == v1   # failed load keeps the old table
+    finally:
+        w8.w8_clear_table()
+    assert w8.w8_gemm_resolve_variant(0, 8, 4096, 4096) != v1

@@ -1,0 +1,95 @@
+"""GPU parity of the quantizers and fused producers against the CPU oracle: codes and
+scales must match bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_gemm_token_b200 import synth, w8
+from gpu_helpers import bits, u8
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("qfmt", [w8.W8_Q_FP8, w8.W8_Q_INT8])
+@pytest.mark.parametrize("M,K", [(1, 8), (1, 1024), (3, 4096), (16, 4096), (32, 12288), (7, 25600),
+                                 (257, 1024), (2, 32768), (5, 136)])
+def test_per_token_bit_exact(orc, qfmt, M, K):
+    x = synth.activations(M, K, seed=1000 + M * 7 + K)
+    q, s = w8.w8_quant_per_token(x.cuda(), qfmt)
+    torch.cuda.synchronize()
+    oq, os_ = orc.quant_rows(qfmt, bits(x))
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq.view(np.uint8))
+
+
+def test_per_token_strided_and_zero_rows(orc):
+    M, K = 6, 1024
+    big = synth.activations(M, K + 64, seed=77)
+    big[2] = 0.0
+    big[4, :] = -0.0
+    xd = big.cuda()[:, :K]
+    for qfmt in (0, 1):
+        q, s = w8.w8_quant_per_token(xd, qfmt)
+        oq, os_ = orc.quant_rows(qfmt, bits(big[:, :K].contiguous()))
+        assert np.array_equal(s.cpu().numpy(), os_)
+        assert np.array_equal(u8(q), oq.view(np.uint8))
+        assert os_[2] == 1.0
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("M,K", [(1, 128), (5, 4096), (32, 5120), (17, 25600), (300, 1024)])
+def test_group128_bit_exact(orc, ue8m0, M, K):
+    x = synth.activations(M, K, seed=2000 + M + K)
+    q, s = w8.w8_quant_per_token(x.cuda(), w8.W8_Q_FP8, group=128, ue8m0=ue8m0)
+    oq, os_ = orc.quant_rows(0, bits(x), group=128, ue8m0=ue8m0)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("N,K", [(128, 128), (300, 520), (1024, 4096)])
+def test_weight_block_bit_exact(orc, ue8m0, N, K):
+    w = synth.weights(N, K, seed=3000 + N + K)
+    q, s = w8.w8_quant_weight_block(w.cuda(), ue8m0=ue8m0)
+    oq, os_ = orc.quant_weight_block(bits(w), ue8m0=ue8m0)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
+
+
+@pytest.mark.parametrize("M,H", [(1, 4096), (5, 4096), (32, 4096), (300, 1024), (3, 8), (2, 25600)])
+def test_rmsnorm_quant_bit_exact(orc, M, H):
+    x = synth.activations(M, H, seed=4000 + M + H)
+    g = synth.gamma(H, seed=4001 + H)
+    q, s = w8.w8_rmsnorm_quant(x.cuda(), g.cuda(), 1e-6)
+    oq, os_ = orc.rmsnorm_quant(bits(x), bits(g), 1e-6)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
+
+
+@pytest.mark.parametrize("M,I", [(1, 12288), (3, 12288), (32, 12288), (64, 1024), (2, 8), (4, 25600)])
+def test_silu_mul_quant_bit_exact(orc, M, I):
+    xgu = synth.activations(M, 2 * I, seed=5000 + M + I)
+    q, s = w8.w8_silu_mul_quant(xgu.cuda())
+    oq, os_ = orc.silu_mul_quant(bits(xgu))
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
+
+
+def test_silu_mul_quant_extreme_gates(orc):
+    I = 64
+    g = torch.linspace(-120, 120, I).to(torch.bfloat16)
+    u = torch.linspace(3, -3, I).to(torch.bfloat16)
+    xgu = torch.cat([g, u])[None, :].repeat(2, 1)
+    q, s = w8.w8_silu_mul_quant(xgu.cuda())
+    oq, os_ = orc.silu_mul_quant(bits(xgu))
+    assert np.array_equal(s.cpu().numpy(), os_) and np.array_equal(u8(q), oq)
+
+
+def test_quant_prefill_rows(orc):
+    """Config-5 prefill activation shape (4096 x 4096), rows checked in full."""
+    M, K = 4096, 4096
+    x = synth.activations(M, K, seed=6000)
+    q, s = w8.w8_quant_per_token(x.cuda(), 0)
+    oq, os_ = orc.quant_rows(0, bits(x))
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
