@@ -1,0 +1,499 @@
+"""Benchmark of the 8-bit quantized linear layer on B200.
+
+Workload (one "step"): the FP8-dynamic decode sweep -- M in {1, 2, 4, 8, 16, 32} tokens
+over the four dense-decoder linear shapes (K x N) 4096x6144 (qkv), 4096x4096 (o_proj),
+4096x24576 (gate_up), 12288x4096 (down).  For each (M, shape): dynamic per-token fp8
+quantization of the bf16 activations, then the scaled FP8 GEMM against per-channel
+e4m3 weights -> bf16 out.  48 launches per step, replayed from one CUDA graph.
+
+Metric: achieved HBM TB/s = algorithmic bytes of the step / step time, where a GEMM
+moves N*K (weights) + M*K (codes) + 4N + 4M (scales) + 2MN (out) bytes and a quantizer
+2MK + MK + 4M.  Weights exist in two copies used alternately (386 MB in total, 3x the
+126 MB L2), so no weight matrix is re-read from L2 between its uses.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--detail] [--single KxN --m M]
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU (the layer
+does not shard: replicas only); value = bytes of all ranks / max-over-ranks time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "8-bit GEMM achieved HBM TB/s and % roofline at M=1-32, Qwen3-like shapes"
+SHAPES = [(4096, 6144), (4096, 4096), (4096, 24576), (12288, 4096)]   # (K, N)
+MS = [1, 2, 4, 8, 16, 32]
+WORKLOAD = ("FP8-dynamic decode sweep: per-token e4m3 quant + scaled GEMM, M in {1,2,4,8,16,32} x "
+            "(KxN) 4096x6144 qkv, 4096x4096 o_proj, 4096x24576 gate_up, 12288x4096 down")
+NCOPY = 2
+
+
+def gemm_bytes(M, N, K):
+    return N * K + M * K + 4 * N + 4 * M + 2 * M * N
+
+
+def quant_bytes(M, K):
+    return 2 * M * K + M * K + 4 * M
+
+
+def step_bytes(shapes=SHAPES, ms=MS):
+    g = sum(gemm_bytes(M, N, K) for M in ms for (K, N) in shapes)
+    q = sum(quant_bytes(M, K) for M in ms for (K, N) in shapes)
+    return g, q
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def gemm_source_hash():
+    h = hashlib.sha256()
+    for f in ("w8_gemm.cu", "w8_ptx.cuh"):
+        with open(os.path.join(ROOT, "bit_quantized_gemm_token_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when the
+    summary is missing or was taken on a different GEMM source."""
+    p = os.path.join(ROOT, "profiles", "gemm_fp8_decode_sweep_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    if d.get("gemm_source_sha") != gemm_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Workload:
+    def __init__(self, dev, shapes, ms, seed, ncopy=NCOPY):
+        import torch
+        from bit_quantized_gemm_token_b200 import w8
+        self.w8 = w8
+        self.shapes, self.ms = shapes, ms
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        self.W = {}   # (shape, copy) -> (Wq, sW)
+        for (K, N) in shapes:
+            for c in range(ncopy):
+                wb = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+                self.W[(K, N, c)] = w8.w8_quant_per_token(wb, w8.W8_Q_FP8)   # per-output-channel
+                del wb
+        self.X, self.A, self.OUT = {}, {}, {}
+        for M in ms:
+            for (K, N) in shapes:
+                x = torch.randn(M, K, device=dev, generator=g)
+                n = M * K
+                idx = torch.randint(0, n, (max(1, n // 1000),), device=dev, generator=g)
+                x.view(-1)[idx] *= 20.0
+                self.X[(M, K, N)] = x.to(torch.bfloat16)
+                self.A[(M, K, N)] = (torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
+                                     torch.empty((M,), dtype=torch.float32, device=dev))
+                self.OUT[(M, K, N)] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        nb = max(w8.w8_gemm_workspace_size(w8.W8_FMT_FP8_DYN, M, N, K, w8.W8_V_PDL)
+                 for M in ms for (K, N) in shapes)
+        self.ws = w8.Workspace(dev, nb)
+        torch.cuda.synchronize()
+
+    def rotate(self, ncopy):
+        """GEMMs of the first (M, shape) against every weight copy in turn."""
+        w8 = self.w8
+        M, (K, N) = self.ms[0], self.shapes[0]
+        q, s = self.A[(M, K, N)]
+        w8.w8_quant_per_token(self.X[(M, K, N)], w8.W8_Q_FP8, q=q, scale=s)
+        for c in range(ncopy):
+            Wq, sW = self.W[(K, N, c)]
+            w8.w8_gemm(w8.W8_FMT_FP8_DYN, q, s, Wq, sW, out=self.OUT[(M, K, N)],
+                       variant=w8.W8_VARIANT_AUTO | w8.W8_V_PDL, workspace=self.ws)
+        return ncopy
+
+    def order(self):
+        for mi, M in enumerate(self.ms):
+            for si, (K, N) in enumerate(self.shapes):
+                yield M, K, N, (mi + si) % NCOPY
+
+    def step(self, quant=True, gemm=True):
+        w8 = self.w8
+        v = w8.W8_VARIANT_AUTO | w8.W8_V_PDL
+        n = 0
+        for M, K, N, c in self.order():
+            q, s = self.A[(M, K, N)]
+            if quant:
+                w8.w8_quant_per_token(self.X[(M, K, N)], w8.W8_Q_FP8, q=q, scale=s)
+                n += 1
+            if gemm:
+                Wq, sW = self.W[(K, N, c)]
+                w8.w8_gemm(w8.W8_FMT_FP8_DYN, q, s, Wq, sW, out=self.OUT[(M, K, N)], variant=v, workspace=self.ws)
+                n += 1
+        return n
+
+
+def time_graph(fn, steps, warmup, world):
+    """Capture fn() into a CUDA graph, replay `warmup` times, then time `steps` replays
+    with CUDA events on the capturing stream.  Returns (ms per step, launches per step)."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()                      # eager warm-up (module load, smem attributes)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        launches = fn()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(steps):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    barrier(world)
+    del g
+    return ms, launches
+
+
+def time_e2e(wl, steps, warmup, world):
+    """Same step through the public API with host buffers: every step copies each
+    activation from pinned host memory to the device, quantizes, multiplies and copies
+    each result back to pinned host memory (events on the stream around all of it)."""
+    import torch
+    w8 = wl.w8
+    s = torch.cuda.Stream()
+    hx = {k: v.cpu().pin_memory() for k, v in wl.X.items()}
+    ho = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in wl.OUT.items()}
+    dx = {k: torch.empty_like(v) for k, v in wl.X.items()}
+    h2d = sum(t.numel() * t.element_size() for t in hx.values())
+    d2h = sum(t.numel() * t.element_size() for t in ho.values())
+    v = w8.W8_VARIANT_AUTO
+
+    def one():
+        for M, K, N, c in wl.order():
+            key = (M, K, N)
+            dx[key].copy_(hx[key], non_blocking=True)
+            q, sc = w8.w8_quant_per_token(dx[key], w8.W8_Q_FP8, q=wl.A[key][0], scale=wl.A[key][1])
+            Wq, sW = wl.W[(K, N, c)]
+            w8.w8_gemm(w8.W8_FMT_FP8_DYN, q, sc, Wq, sW, out=wl.OUT[key], variant=v, workspace=wl.ws)
+            ho[key].copy_(wl.OUT[key], non_blocking=True)
+
+    with torch.cuda.stream(s):
+        for _ in range(warmup):
+            one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(steps):
+            one()
+        e1.record(s)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+class OracleSample:
+    """The CPU oracle as it stands (single-threaded C, fp64 GEMM) on a bounded sample of
+    the same workload: for every (M, shape) pair, per-token quantization of the full
+    activations and the first `cols` output columns of the GEMM.  Throughput is given in
+    the metric's unit: algorithmic bytes of the sampled work (weight rows of the
+    sampled columns, codes, scales, outputs, quantizer traffic) / time."""
+
+    def __init__(self, shapes, ms):
+        import oracle as orc
+        from bit_quantized_gemm_token_b200 import synth
+        self.orc = orc
+        self.shapes, self.ms = shapes, ms
+        self.data = {}
+        for (K, N) in shapes:
+            w = synth.weights(1024, K, seed=synth.SEED_BASE + 2 + N)
+            wq, ws = orc.quant_rows(0, synth.bf16_bits(w))
+            for M in ms:
+                x = synth.activations(M, K, seed=synth.SEED_BASE + 2 + M * 100 + K)
+                self.data[(M, K, N)] = (synth.bf16_bits(x), wq, ws)
+        self.cols = 64
+
+    def run(self):
+        nbytes = 0
+        t0 = time.perf_counter()
+        for M in self.ms:
+            for (K, N) in self.shapes:
+                xb, wq, ws = self.data[(M, K, N)]
+                aq, sa = self.orc.quant_rows(0, xb)
+                self.orc.gemm(0, aq, sa, wq[:self.cols], ws[:self.cols])
+                nbytes += quant_bytes(M, K) + gemm_bytes(M, self.cols, K)
+        return nbytes, time.perf_counter() - t0
+
+    def size_for(self, seconds):
+        """Grow the column sample until one run takes about `seconds`."""
+        nb, dt = self.run()
+        if dt < seconds:
+            self.cols = int(min(1024, max(self.cols, self.cols * seconds / max(dt, 1e-3))))
+            nb, dt = self.run()
+        return nb, dt
+
+    def describe(self, dt):
+        return ("all %d (M, shape) pairs of the workload: per-token quant of the full activations + the first "
+                "%d output columns of each GEMM (fp64 triple loop); %.1f s per sample"
+                % (len(self.ms) * len(self.shapes), self.cols, dt))
+
+
+def cpu_baseline(shapes, ms, target_s=10.0):
+    smp = OracleSample(shapes, ms)
+    nb, dt = smp.size_for(target_s)
+    return {"value": nb / dt / 1e12, "unit": "TB/s", "cores": 1, "kind": "oracle", "sample": smp.describe(dt)}
+
+
+def run_ours(args):
+    import torch
+    from bit_quantized_gemm_token_b200 import w8
+    w8.lib()   # raises if the CUDA library is not built: there is no fallback
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    shapes, ms = SHAPES, MS
+    workload = WORKLOAD
+    if args.single:
+        K, N = (int(v) for v in args.single.lower().split("x"))
+        shapes, ms = [(K, N)], [args.m]
+        workload = "single FP8-dynamic quant + GEMM, M=%d, KxN=%dx%d" % (args.m, K, N)
+    wl = Workload(dev, shapes, ms, seed=1234 + 1 + rank)
+    gb, qb = step_bytes(shapes, ms)
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(torch.cuda.current_device())
+    clk = ClockSampler(gpu_id) if rank == 0 and not args.no_clocks else None
+    if clk:
+        clk.start()
+    ms_step, launches = time_graph(lambda: wl.step(True, True), args.steps, args.warmup, world)
+    ms_gemm, n_gemm = time_graph(lambda: wl.step(False, True), args.steps, args.warmup, world)
+    clocks = clk.stop() if clk else None
+    ms_step = max_over_ranks(world, ms_step)
+    ms_gemm = max_over_ranks(world, ms_gemm)
+
+    e2e = None
+    if not args.no_e2e:
+        ms_e2e, h2d, d2h = time_e2e(wl, max(1, args.steps // 2), max(1, args.warmup // 2), world)
+        ms_e2e = max_over_ranks(world, ms_e2e)
+        e2e = {"value": round(world * (gb + qb) / (ms_e2e * 1e-3) / 1e12, 4), "unit": "TB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4),
+               "path": "w8_quant_per_token + w8_gemm (AUTO) eagerly, pinned host buffers"}
+
+    detail = None
+    if args.detail and rank == 0:
+        detail = []
+        for (K, N) in shapes:
+            for M in ms:
+                ncopy = max(2, -(-400_000_000 // (N * K)))     # > 3x L2 of weights in rotation
+                sub = Workload(dev, [(K, N)], [M], seed=99, ncopy=ncopy)
+                t, nl = time_graph(lambda: sub.rotate(ncopy), 5, 3, 1)
+                t /= nl
+                b = gemm_bytes(M, N, K)
+                detail.append({"K": K, "N": N, "M": M, "us": round(t * 1e3, 2), "TB/s": round(b / (t * 1e-3) / 1e12, 3),
+                               "variant": w8.describe(w8.w8_gemm_resolve_variant(0, M, N, K))})
+                del sub
+
+    peak, peak_kind = load_peaks()
+    achieved = gb / (ms_gemm * 1e-3) / 1e9    # GB/s, GEMM kernels alone
+    n_gemm_per_step = len(shapes) * len(ms)
+    traffic = traffic_from_profile()
+    value = world * (gb + qb) / (ms_step * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 4), "unit": "TB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": workload, "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: %d weight copies per shape used alternately (%.0f MB of weights)"
+                         % (NCOPY, sum(N * K for (K, N) in shapes) * NCOPY / 1e6),
+                   "launch": "CUDA graph of the step; GEMM variant AUTO + programmatic dependent launch",
+                   "bytes_per_step": gb + qb},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                     "traffic": (round(traffic) if traffic is not None else None),
+                     "algorithmic_bytes_per_launch": round(gb / n_gemm_per_step),
+                     "kernel": "gemm_kernel (w8_gemm FP8-dynamic)", "ms_gemm_per_step": round(ms_gemm, 4),
+                     "frac_of_8TBs": round(achieved / 8000.0, 4)},
+        "gpu_launches": launches * args.steps,
+    }
+    if clocks:
+        out["clocks"] = clocks
+    if e2e:
+        out["e2e"] = e2e
+    if detail:
+        out["detail"] = detail
+    if rank == 0 and world == 1 and not args.no_cpu:
+        out["cpu_baseline"] = cpu_baseline(shapes, ms, target_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The reference arm is the CPU oracle as it stands (the pages ship no runnable
+    code): each step is one bounded sample of the same workload on the host cores, in
+    the same metric and unit.  Under torchrun only rank 0 runs and prints."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    smp = OracleSample(SHAPES, MS)
+    smp.size_for(max(0.5, args.ref_seconds))       # sizing run (counts as warm-up)
+    for _ in range(max(0, args.warmup - 1)):
+        smp.run()
+    tot_b, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        nb, dt = smp.run()
+        tot_b += nb
+        tot_t += dt
+    val = tot_b / tot_t / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": round(val, 9), "unit": "TB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "parallelism": "one host thread"},
+           "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": smp.describe(tot_t / args.steps),
+                            "value": round(val, 9), "unit": "TB/s"},
+           "e2e": {"value": round(val, 9), "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--detail", action="store_true", help="also time every (shape, M) GEMM alone")
+    ap.add_argument("--single", default="", help="KxN: time one shape only (profiling case)")
+    ap.add_argument("--m", type=int, default=32)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=3.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,714 @@
+// w8_gemm_kernel.cuh -- the scaled 8-bit GEMM kernel template: one sm_100a kernel family (tcgen05 MMA, TMEM
+// accumulators, TMA shared-memory pipeline) whose Standard, Split-K and Swap-AB forms
+// are run-time choices, for FP8-dynamic, W8A8-INT8 and Block-FP8.
+//
+// What it computes ("Helion DSL added to vLLM to autotune linear inference backends",
+// section "Unified GEMM Architecture"; "Helion nel backend vLLM: un solo GEMM ...",
+// paragraphs 2-3; "PyTorch integra Helion en vLLM para acelerar inferencia FP8",
+// section "Kernels Helion implementados": scaled_mm, scaled_mm_blockwise):
+//   FP8_DYN  out[m,n] = bf16( sum_k A[m,k] W[n,k] * sA[m] * sW[n] ), fp32 accumulation
+//   INT8     out[m,n] = bf16( float(sum_k A W as int32) * sA[m] * sW[n] )
+//   BLOCK    out[m,n] = bf16( sum_kb sA[m,kb] sW[n/128,kb] sum_{k in kb} A W )
+//
+// Structure.  Both operands are K-major byte matrices.  The MMA's 128-row operand "R"
+// and its BN-row operand "C" are bound at launch: Standard binds R = A (tokens) and
+// C = W; Swap-AB binds R = W and C = A, so the accumulator is out^T and the epilogue
+// writes the transpose (the pages' A@B = (B^T A^T)^T).  The problem is cut into units
+// (output tile, 128-column K block).  CTA g owns the contiguous unit range
+// [g*U/G, (g+1)*U/G): with G = tiles * split_k each CTA holds one 1/split_k K-chunk of
+// one tile (Split-K); with G = the SM count the units are dealt out evenly (a
+// balanced split); with whole-tile ranges nothing is split (Standard).  A tile whose K
+// range is shared by several CTAs is finished by whichever arrives last (an atomic
+// ticket, no waiting): it adds the fp32 (int32 for INT8) partials of the contributors
+// in CTA order, which fixes the summation order, applies the scales and stores bf16.
+//
+// Per CTA (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer
+// (one elected lane), warps 2..5 = epilogue (TMEM -> registers -> scales -> global).
+// Shared memory holds `stages` (R, C) tile pairs, 128-byte swizzled, behind full/empty
+// mbarriers; the accumulator is double-buffered in TMEM (tfull/tempty mbarriers) so
+// the epilogue of one tile overlaps the MMAs of the next.  Block-FP8 hands each
+// 128-column K block to the epilogue, which scales it and accumulates in fp32
+// registers.  Every wait is bounded by the global timer; on expiry the CTA records
+// W8_ERR_DEVICE_TIMEOUT in the device status word, unwinds and frees its TMEM.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "w8_internal.h"
+#include "w8_ptx.cuh"
+
+namespace w8 {
+namespace gemm {
+
+// first device-side error (0 = none); one word per translation unit that instantiates
+// kernels, read through that unit's status accessor
+static __device__ int g_device_status;
+
+
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kEpiBarrier = 1;          // named barrier id of the epilogue warps
+constexpr int kTmemBarrier = 2;         // named barrier id of warps 1..5 (TMEM hand-off)
+constexpr int kNumAcc = 2;              // TMEM accumulator buffers
+constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s bound on any single wait
+constexpr int kL2Ahead = 6;             // units whose weights are prefetched to L2 before the PDL wait
+
+enum { KIND_F8 = 0, KIND_I8 = 1 };
+
+struct GemmArgs {
+    int M, N, K;
+    int swap;
+    int rows_R, rows_C;
+    int r_tiles, c_tiles, tiles;
+    int kbs;   // 128-column K blocks
+    int nsb;   // stage blocks (units) per tile = ceil(kbs / KPS)
+    long long units;
+    int G;
+    int align_tiles;
+    int stages;
+    int pdl;
+    int ld_sblk;   // K/128: row length of the block-scale matrices
+    int vec_ok;    // Standard epilogue may use 16-byte stores (N % 8 == 0, out 16-byte aligned)
+    int csplit;    // cluster split: the K chunks of a tile are the CTAs of one cluster (0 = off)
+    const uint8_t* w_ptr;   // weight codes [N, K] (for the L2 prefetch under PDL)
+    const float* sA;
+    const float* sW;
+    __nv_bfloat16* out;
+    int32_t* out_i32;
+    uint32_t* partials;   // [G][2][BN][128] raw fp32 / int32 words
+    int* counters;        // [tiles]
+};
+
+// ---------------------------------------------------------------- descriptors
+// Shared-memory matrix descriptor (tcgen05): K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row core-matrix groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);   // bits 0-13: start address >> 4
+    d |= (uint64_t)(16u >> 4) << 16;             // bits 16-29: leading byte offset (unused here)
+    d |= (uint64_t)(1024u >> 4) << 32;           // bits 32-45: stride byte offset
+    d |= (uint64_t)1 << 46;                      // bits 46-47: descriptor version 1
+    d |= (uint64_t)2 << 61;                      // bits 61-63: 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor: dense, D = f32 (e4m3 x e4m3) or s32 (s8 x s8), both operands
+// K-major, M = BM (64 or 128), N = BN.
+template <int KIND, int BM, int BN>
+__device__ __forceinline__ constexpr uint32_t instr_desc()
+{
+    return (KIND == KIND_I8 ? (2u << 4) : (1u << 4))      // bits 4-5: D format
+           | (KIND == KIND_I8 ? (1u << 7) : 0u)           // bits 7-9: A format (s8 / e4m3)
+           | (KIND == KIND_I8 ? (1u << 10) : 0u)          // bits 10-12: B format
+           | ((uint32_t)(BN >> 3) << 17)                  // bits 17-22: N / 8
+           | ((uint32_t)(BM >> 4) << 24);                 // bits 24-28: M / 16
+}
+
+// ---------------------------------------------------------------- unit partition
+__device__ __forceinline__ long long unit_begin(const GemmArgs& a, long long g)
+{
+    if (a.align_tiles) return (g * a.tiles / a.G) * a.nsb;
+    return g * a.units / a.G;
+}
+
+__device__ __forceinline__ int cta_of_unit(const GemmArgs& a, long long u)
+{
+    return (int)(((u + 1) * (long long)a.G - 1) / a.units);
+}
+
+// ---------------------------------------------------------------- bounded waits
+__device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_status, 0, code); }
+
+// Poll an mbarrier phase until it completes, the deadline passes, or another role of
+// this CTA has given up (abort flag).  Returns false on give-up.
+template <bool CLUSTER_SCOPE = false>
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag)
+{
+    auto probe = [&] { return CLUSTER_SCOPE ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity); };
+    if (probe()) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (probe()) return true;
+        if ((it & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer_ns() - t0 > kWaitNs) {
+                *abort_flag = 1;
+                record_error(W8_ERR_DEVICE_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- epilogue helpers
+template <int KIND>
+__device__ __forceinline__ float word_to_float(uint32_t w)
+{
+    return KIND == KIND_I8 ? (float)(int32_t)w : __uint_as_float(w);
+}
+
+template <int KIND>
+__device__ __forceinline__ uint32_t add_words(uint32_t x, uint32_t y)
+{
+    return KIND == KIND_I8 ? (uint32_t)((int32_t)x + (int32_t)y) : __float_as_uint(__fadd_rn(__uint_as_float(x), __uint_as_float(y)));
+}
+
+// Store one output element (row i of the R tile, column j of the C tile).  `w` is the
+// raw accumulator word: unscaled (FP8/INT8) or already block-scaled (BLOCK).
+template <int KIND, bool BLOCK>
+__device__ __forceinline__ void store_out(const GemmArgs& a, int r_row, int c_row, uint32_t w, float s_row)
+{
+    const int m = a.swap ? c_row : r_row;
+    const int n = a.swap ? r_row : c_row;
+    if (m >= a.M || n >= a.N) return;
+    const size_t o = (size_t)m * a.N + n;
+    if (KIND == KIND_I8 && a.out_i32 != nullptr) {
+        a.out_i32[o] = (int32_t)w;
+        return;
+    }
+    float v = word_to_float<KIND>(w);
+    if (!BLOCK) {
+        // s_row is the scale of the R-side index; the C-side scale is looked up here
+        const float s_col = a.swap ? __ldg(a.sA + m) : __ldg(a.sW + n);
+        v = a.swap ? __fmul_rn(__fmul_rn(v, s_col), s_row) : __fmul_rn(__fmul_rn(v, s_row), s_col);
+    }
+    a.out[o] = __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Store 16 consecutive C-tile columns [c_base, c_base + 16) of R-tile row r_row.  In the
+// Standard form these are 16 consecutive outputs of one row: two 16-byte stores.
+template <int KIND, bool BLOCK>
+__device__ __forceinline__ void store_chunk16(const GemmArgs& a, int r_row, int c_base, const uint32_t (&v)[16],
+                                              float s_row)
+{
+    if (!a.swap && a.vec_ok && a.out_i32 == nullptr && r_row < a.M && c_base + 15 < a.N) {
+        float f[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+            f[jj] = word_to_float<KIND>(v[jj]);
+            if (!BLOCK) f[jj] = __fmul_rn(__fmul_rn(f[jj], s_row), __ldg(a.sW + c_base + jj));
+        }
+        uint4 lo, hi;
+        lo.x = pack_bf16x2(f[0], f[1]);   lo.y = pack_bf16x2(f[2], f[3]);
+        lo.z = pack_bf16x2(f[4], f[5]);   lo.w = pack_bf16x2(f[6], f[7]);
+        hi.x = pack_bf16x2(f[8], f[9]);   hi.y = pack_bf16x2(f[10], f[11]);
+        hi.z = pack_bf16x2(f[12], f[13]); hi.w = pack_bf16x2(f[14], f[15]);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + (size_t)r_row * a.N + c_base);
+        dst[0] = lo;
+        dst[1] = hi;
+        return;
+    }
+#pragma unroll
+    for (int jj = 0; jj < 16; ++jj) store_out<KIND, BLOCK>(a, r_row, c_base + jj, v[jj], s_row);
+}
+
+// ---------------------------------------------------------------- the kernel
+// BM = rows of the MMA's M operand ("R": 128, or 64 for a narrow token tile), BN = rows
+// of its N operand ("C"), KPS = 128-column K blocks per pipeline stage (1 or 2).  A
+// "unit" of the partition is one stage block of KPS K blocks of one output tile.
+// Accumulator row r of a BM = 64 MMA lives in TMEM lane (r % 16) + 32 * (r / 16); of a
+// BM = 128 MMA in lane r.
+template <int BM, int BN, int KIND, bool BLOCK, int KPS>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC, const GemmArgs a)
+{
+    constexpr int kRBytes = BM * 128;
+    constexpr int kCBytes = BN * 128;
+    constexpr int kStageBytes = KPS * (kRBytes + kCBytes);
+    constexpr uint32_t kTmemCols = (kNumAcc * BN <= 32) ? 32 : (kNumAcc * BN <= 64) ? 64 : (kNumAcc * BN <= 128) ? 128 : (kNumAcc * BN <= 256) ? 256 : 512;
+    constexpr uint32_t kIdesc = instr_desc<KIND, BM, BN>();
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = a.stages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * kStageBytes);
+    uint64_t* empty = full + S;
+    uint64_t* tfull = empty + S;
+    uint64_t* tempty = tfull + kNumAcc;
+    uint64_t* drain = tempty + kNumAcc;
+    uint64_t* red_full = drain + 1;   // cluster split: partials of the other ranks have landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* ticket = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    // cluster split: [csplit - 1][BN columns][128 rows] partial words, used in rank 0 only
+    uint32_t* red_buf = reinterpret_cast<uint32_t*>(tmem_slot + 4);
+    // stage s: R slots [KPS][128 x 128 B], then C slots [KPS][BN x 128 B]; all 1024-aligned
+    auto r_slot = [&](int s, int j) { return smem + (size_t)s * kStageBytes + (size_t)j * kRBytes; };
+    auto c_slot = [&](int s, int j) { return smem + (size_t)s * kStageBytes + (size_t)KPS * kRBytes + (size_t)j * kCBytes; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(ptx::smem_u32(full + s), 1);
+            ptx::mbar_init(ptx::smem_u32(empty + s), 1);
+        }
+        for (int b = 0; b < kNumAcc; ++b) {
+            ptx::mbar_init(ptx::smem_u32(tfull + b), 1);
+            ptx::mbar_init(ptx::smem_u32(tempty + b), kEpiThreads / 32);
+        }
+        ptx::mbar_init(ptx::smem_u32(drain), 1);
+        ptx::mbar_init(ptx::smem_u32(red_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * kEpiThreads : 1u);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        ptx::prefetch_tmap(&tmR);
+        ptx::prefetch_tmap(&tmC);
+    }
+    __syncthreads();
+    // cluster split: rank 0's reduction barrier must be initialised before any other
+    // rank can arrive on it
+    if (a.csplit > 1) ptx::cluster_sync();
+    // TMEM is allocated by warp 1 and handed to warps 1..5 through a named barrier, so
+    // the producer can start streaming while the allocation still waits for columns a
+    // CTA of the previous kernel holds
+    uint32_t tmem = 0;
+    if (warp != 0) {
+        if (warp == 1) ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+        ptx::tc_fence_before();
+        ptx::bar_sync(kTmemBarrier, kThreads - 32);
+        ptx::tc_fence_after();
+        tmem = *tmem_slot;
+    }
+
+    const long long u0 = unit_begin(a, blockIdx.x);
+    const long long u1 = unit_begin(a, blockIdx.x + 1);
+    const int nsb = a.nsb;   // stage blocks per tile
+    const int kbs = a.kbs;   // 128-column K blocks per tile
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t pol_w = ptx::policy_evict_first();   // weights: streamed once
+            const uint64_t pol_a = ptx::policy_evict_last();    // activations: re-read by every CTA
+            const uint64_t pol_R = a.swap ? pol_w : pol_a;
+            const uint64_t pol_C = a.swap ? pol_a : pol_w;
+            const long long n = u1 - u0;
+            // load the R boxes (load_r) and/or C boxes of unit u into stage s
+            auto issue = [&](int s, long long u, bool load_r, bool load_c, bool expect) {
+                const int t = (int)(u / nsb), kb0 = (int)(u % nsb) * KPS;
+                const int nkb = (kbs - kb0 < KPS) ? kbs - kb0 : KPS;
+                const int rt = t / a.c_tiles, ct = t % a.c_tiles;
+                const uint32_t fb = ptx::smem_u32(full + s);
+                if (expect) ptx::mbar_arrive_expect_tx(fb, (uint32_t)(nkb * (kRBytes + kCBytes)));
+                for (int j = 0; j < nkb; ++j) {
+                    if (load_r) ptx::tma_load_2d(ptx::smem_u32(r_slot(s, j)), &tmR, fb, (kb0 + j) * 128, rt * BM, pol_R);
+                    if (load_c) ptx::tma_load_2d(ptx::smem_u32(c_slot(s, j)), &tmC, fb, (kb0 + j) * 128, ct * BN, pol_C);
+                }
+            };
+            // With programmatic dependent launch this kernel releases its dependents at
+            // once and, before waiting for the kernels ahead of it, requests the weight
+            // boxes of the first `pre` stages (weights are never the output of work in
+            // flight; the epilogue warps prefetch the next units' weights into L2); the
+            // activation boxes follow after the wait.
+            ptx::grid_dep_launch();
+            const int pre = a.pdl ? (int)(n < S ? n : S) : 0;
+            for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap != 0, a.swap == 0, true);
+            ptx::grid_dep_wait();
+            for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap == 0, a.swap != 0, false);
+            long long issued = pre;
+            int stage = pre % S;
+            uint32_t phase = (pre == S) ? 1u : 0u;
+            for (long long i = pre; i < n; ++i) {
+                if (!wait_bounded(ptx::smem_u32(empty + stage), phase ^ 1u, abort_flag)) break;
+                issue(stage, u0 + i, true, true, true);
+                ++issued;
+                if (++stage == S) { stage = 0; phase ^= 1u; }
+            }
+            if (*abort_flag) {
+                // let the copies still in flight land before the CTA unwinds: the last
+                // min(S, issued) stages (earlier ones were consumed), each bounded
+                const long long lo = issued > S ? issued - S : 0;
+                for (long long j = lo; j < issued; ++j) {
+                    const uint32_t fb = ptx::smem_u32(full + (int)(j % S));
+                    const uint32_t par = (uint32_t)((j / S) & 1);
+                    const uint64_t t0 = ptx::globaltimer_ns();
+                    while (!ptx::mbar_try_wait(fb, par) && ptx::globaltimer_ns() - t0 < 10000000ull) {}
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // (its bounded waits start only once the kernels ahead of this one are done)
+        ptx::grid_dep_wait();
+        int stage = 0, buf = 0;
+        uint32_t phase = 0, bphase = 0;
+        bool ok = true;
+        for (long long u = u0; u < u1 && ok; ++u) {
+            const int sb = (int)(u % nsb);
+            const int kb0 = sb * KPS;
+            const int nkb = (kbs - kb0 < KPS) ? kbs - kb0 : KPS;
+            const bool seg_first = (u == u0 || sb == 0);
+            const bool seg_last = (u == u1 - 1 || sb == nsb - 1);
+            int nbuf_used = 0;
+            if (lane == 0) {
+                if (!BLOCK && seg_first) {
+                    ok = wait_bounded(ptx::smem_u32(tempty + buf), bphase ^ 1u, abort_flag);
+                    ptx::tc_fence_after();
+                }
+                if (ok) ok = wait_bounded(ptx::smem_u32(full + stage), phase, abort_flag);
+                if (ok) {
+                    ptx::tc_fence_after();
+                    int b = buf;
+                    uint32_t bp = bphase;
+                    for (int j = 0; j < nkb && ok; ++j) {
+                        if (BLOCK) {
+                            // every K block gets its own accumulator, handed to the epilogue
+                            ok = wait_bounded(ptx::smem_u32(tempty + b), bp ^ 1u, abort_flag);
+                            ptx::tc_fence_after();
+                            if (!ok) break;
+                        }
+                        const uint64_t dR = smem_desc(ptx::smem_u32(r_slot(stage, j)));
+                        const uint64_t dC = smem_desc(ptx::smem_u32(c_slot(stage, j)));
+                        const uint32_t d_tmem = tmem + (uint32_t)(b * BN);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            // advance 32 K-bytes inside the 128-byte swizzle row: +2 in 16-byte units
+                            const uint32_t acc = BLOCK ? (k > 0 ? 1u : 0u) : ((seg_first && j == 0 && k == 0) ? 0u : 1u);
+                            if (KIND == KIND_I8) ptx::mma_i8(d_tmem, dR + 2 * k, dC + 2 * k, kIdesc, acc);
+                            else                 ptx::mma_f8f6f4(d_tmem, dR + 2 * k, dC + 2 * k, kIdesc, acc);
+                        }
+                        if (BLOCK) {
+                            ptx::mma_commit(ptx::smem_u32(tfull + b));
+                            if (++b == kNumAcc) { b = 0; bp ^= 1u; }
+                            ++nbuf_used;
+                        }
+                    }
+                    if (ok) {
+                        ptx::mma_commit(ptx::smem_u32(empty + stage));
+                        if (!BLOCK && seg_last) ptx::mma_commit(ptx::smem_u32(tfull + buf));
+                    }
+                }
+            }
+            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+            nbuf_used = __shfl_sync(0xFFFFFFFFu, nbuf_used, 0);
+            if (++stage == S) { stage = 0; phase ^= 1u; }
+            if (BLOCK) {
+                for (int j = 0; j < nbuf_used; ++j)
+                    if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+            } else if (seg_last) {
+                if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+            }
+        }
+        if (!ok && lane == 0) {
+            // MMAs already issued must finish before TMEM is released (bounded)
+            ptx::mma_commit(ptx::smem_u32(drain));
+            const uint64_t t0 = ptx::globaltimer_ns();
+            while (!ptx::mbar_try_wait(ptx::smem_u32(drain), 0) && ptx::globaltimer_ns() - t0 < 10000000ull) {}
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        if (a.pdl) {
+            // Idle until the first accumulator is ready: prefetch into L2 the weight rows
+            // of the kL2Ahead units that follow the producer's first stages, so that the
+            // weight stream keeps HBM busy while the kernels ahead of this one finish.
+            const long long p0 = u0 + S, p1 = (u1 < p0 + kL2Ahead) ? u1 : p0 + kL2Ahead;
+            const int wrows = a.swap ? BM : BN;
+            const int lines_per_row = KPS;                  // 128-byte lines per row per unit
+            const long long total = (p1 > p0) ? (p1 - p0) * wrows * lines_per_row : 0;
+            for (long long e = threadIdx.x - 64; e < total; e += kEpiThreads) {
+                const long long u = p0 + e / (wrows * lines_per_row);
+                const int rem = (int)(e % (wrows * lines_per_row));
+                const int t = (int)(u / nsb), kb = (int)(u % nsb) * KPS + rem % lines_per_row;
+                const int row = (a.swap ? (t / a.c_tiles) * BM : (t % a.c_tiles) * BN) + rem / lines_per_row;
+                if (row < a.N && kb < kbs) ptx::prefetch_l2_evict_last(a.w_ptr + (size_t)row * a.K + (size_t)kb * 128);
+            }
+        }
+        ptx::grid_dep_wait();
+        const int q = warp & 3;                 // TMEM lane quadrant of this warp
+        // row of the R tile held by this thread (BM = 64: lanes 16..31 of a quadrant hold none)
+        const int i = (BM == 128) ? q * 32 + lane : q * 16 + (lane & 15);
+        const bool lane_has_row = (BM == 128) || lane < 16;
+        const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
+        const bool first_epi = (threadIdx.x == 64);
+        constexpr int kAccRegs = BLOCK ? BN : 1;
+        int buf = 0;
+        uint32_t bphase = 0;
+        bool ok = true;
+        for (long long u = u0; u < u1 && ok;) {
+            const int t = (int)(u / nsb);
+            const int sb_lo = (int)(u % nsb);
+            const long long rem = u1 - u;
+            const int sb_hi = (int)((nsb - sb_lo < rem) ? nsb : sb_lo + rem);
+            const int rt = t / a.c_tiles, ct = t % a.c_tiles;
+            // sentinel for threads holding no real row: padding lanes of the 64-row tile and,
+            // in the Standard form, token rows past M (their accumulators are zero)
+            const int r_row = (lane_has_row && rt * BM + i < a.rows_R) ? rt * BM + i : 0x7FFFFFFF;
+            const bool has_row = r_row != 0x7FFFFFFF;
+            const bool full_tile = (sb_lo == 0 && sb_hi == nsb);
+            const int slot = (u == u0) ? 0 : 1;
+            // scale of this thread's R-side index (FP8 / INT8; BLOCK scales per K block)
+            float s_row = 1.0f;
+            if (!BLOCK && a.out_i32 == nullptr && r_row < a.rows_R) s_row = __ldg((a.swap ? a.sW : a.sA) + r_row);
+
+            float acc[kAccRegs];
+#pragma unroll
+            for (int j = 0; j < kAccRegs; ++j) acc[j] = 0.0f;
+            if (BLOCK) {
+                // ---- per-K-block promotion: acc += (sA * sW) * (block dot product), fp32
+                const int kb_end = (sb_hi * KPS < kbs) ? sb_hi * KPS : kbs;
+                for (int kb = sb_lo * KPS; kb < kb_end; ++kb) {
+                    const bool w = wait_bounded(ptx::smem_u32(tfull + buf), bphase, abort_flag);
+                    if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    // scales of this K block: swap -> sW scalar, sA per column (lane-loaded,
+                    // shuffled); standard -> one product per thread
+                    float sa_l[(BN + 31) / 32];
+                    float sc_thread = 0.0f, sw = 0.0f;
+                    if (a.swap) {
+                        sw = __ldg(a.sW + (size_t)rt * a.ld_sblk + kb);
+#pragma unroll
+                        for (int h = 0; h < (BN + 31) / 32; ++h) {
+                            const int jc = h * 32 + lane;
+                            const int col = ct * BN + jc;
+                            sa_l[h] = (jc < BN && col < a.rows_C) ? __ldg(a.sA + (size_t)col * a.ld_sblk + kb) : 0.0f;
+                        }
+                    } else {
+                        const float sa = (r_row < a.rows_R) ? __ldg(a.sA + (size_t)r_row * a.ld_sblk + kb) : 0.0f;
+                        sc_thread = __fmul_rn(sa, __ldg(a.sW + (size_t)((ct * BN) / 128) * a.ld_sblk + kb));
+                    }
+#pragma unroll
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        uint32_t v[16];
+                        ptx::tmem_ld16(t_lane + (uint32_t)(buf * BN + c0), v);
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) {
+                            const int j = c0 + jj;
+                            const float sc = a.swap ? __fmul_rn(__shfl_sync(0xFFFFFFFFu, sa_l[j / 32], j % 32), sw)
+                                                    : sc_thread;
+                            acc[BLOCK ? j : 0] = __fmaf_rn(__uint_as_float(v[jj]), sc, acc[BLOCK ? j : 0]);
+                        }
+                    }
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(tempty + buf));
+                    if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+                }
+                if (!ok) break;
+            } else {
+                const bool w = wait_bounded(ptx::smem_u32(tfull + buf), bphase, abort_flag);
+                if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) { ok = false; break; }
+                ptx::tc_fence_after();
+            }
+
+            // 16 accumulator words of column chunk c0: from TMEM (FP8/INT8) or registers (BLOCK)
+            auto fetch16 = [&](int c0, uint32_t (&v)[16]) {
+                if (BLOCK) {
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) v[jj] = __float_as_uint(acc[BLOCK ? (c0 + jj) % kAccRegs : 0]);
+                } else {
+                    ptx::tmem_ld16(t_lane + (uint32_t)(buf * BN + c0), v);
+                }
+            };
+
+            // columns of this tile that hold real rows of the C operand (tokens for
+            // Swap-AB: only these are written, published and reduced)
+            const int ncv = (a.rows_C - ct * BN < BN) ? a.rows_C - ct * BN : BN;
+            if (a.csplit > 1) {
+                // ---- cluster split: ranks 1.. write their partial accumulators into rank
+                // 0's shared memory (distributed shared memory) and arrive on its barrier;
+                // rank 0 adds them in rank order, scales and stores
+                const uint32_t rank = ptx::cluster_ctarank();
+                if (rank != 0) {
+                    const uint32_t rbase = ptx::map_to_rank(ptx::smem_u32(red_buf), 0) +
+                                           (rank - 1) * (uint32_t)(BN * BM * 4);
+#pragma unroll
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        if (c0 >= ncv) break;
+                        uint32_t v[16];
+                        fetch16(c0, v);
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (c0 + jj < ncv && has_row) ptx::st_cluster_u32(rbase + (uint32_t)(((c0 + jj) * BM + i) * 4), v[jj]);
+                    }
+                    ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(red_full), 0));
+                } else {
+                    const bool w = wait_bounded<true>(ptx::smem_u32(red_full), 0, abort_flag);
+                    if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) { ok = false; break; }
+#pragma unroll
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        if (c0 >= ncv) break;
+                        uint32_t v[16];
+                        fetch16(c0, v);
+                        for (int r = 1; r < a.csplit; ++r) {
+                            const uint32_t* src = red_buf + (size_t)(r - 1) * (BN * BM);
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                v[jj] = add_words<BLOCK ? KIND_F8 : KIND>(v[jj], src[(c0 + jj) * BM + i]);
+                        }
+                        store_chunk16<KIND, BLOCK>(a, r_row, ct * BN + c0, v, s_row);
+                    }
+                }
+            } else if (full_tile) {
+                // ---- whole K range in this CTA: scale and store
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (c0 >= ncv) break;
+                    uint32_t v[16];
+                    fetch16(c0, v);
+                    store_chunk16<KIND, BLOCK>(a, r_row, ct * BN + c0, v, s_row);
+                }
+            } else {
+                // ---- partial: publish to this CTA's slot ([column][row] words, coalesced)
+                uint32_t* my = a.partials + ((size_t)blockIdx.x * 2 + slot) * (size_t)(BN * BM);
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (c0 >= ncv) break;
+                    uint32_t v[16];
+                    fetch16(c0, v);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        if (c0 + jj < ncv && has_row) __stcg(my + (size_t)(c0 + jj) * BM + i, v[jj]);
+                }
+            }
+            if (!BLOCK) {
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(tempty + buf));
+                if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+            }
+            if (!full_tile && a.csplit <= 1) {
+                // ---- ticket: the last contributor of tile t finishes it
+                __threadfence();
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (first_epi) *ticket = atomicAdd(a.counters + t, 1);
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                const int g_lo = cta_of_unit(a, (long long)t * nsb);
+                const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1);
+                if (*ticket == g_hi - g_lo) {
+                    __threadfence();
+                    const int nc = g_hi - g_lo + 1;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < ncv; c0 += 16) {
+                        uint32_t v[16];
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) v[jj] = 0u;
+                        // contributors four at a time (their loads in flight together),
+                        // added in CTA order, which fixes the summation order
+#pragma unroll 1
+                        for (int cb = 0; cb < nc; cb += 4) {
+                            uint32_t x[4][16];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const int c = g_lo + cb + k;
+                                if (cb + k < nc) {
+                                    const int sl = (unit_begin(a, c) / nsb == t) ? 0 : 1;
+                                    const uint32_t* p = a.partials + ((size_t)c * 2 + sl) * (size_t)(BN * BM);
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj)
+                                        x[k][jj] = (c0 + jj < ncv && has_row) ? __ldcg(p + (size_t)(c0 + jj) * BM + i) : 0u;
+                                }
+                            }
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                if (cb + k < nc) {
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj)
+                                        v[jj] = (cb + k == 0) ? x[k][jj] : add_words<BLOCK ? KIND_F8 : KIND>(v[jj], x[k][jj]);
+                                }
+                            }
+                        }
+                        store_chunk16<KIND, BLOCK>(a, r_row, ct * BN + c0, v, s_row);
+                    }
+                    if (first_epi) a.counters[t] = 0;   // leave the counter ready for the next call
+                }
+            }
+            u += sb_hi - sb_lo;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+
+template <int BM, int BN, int KIND, bool BLOCK, int KPS>
+cudaError_t launch_one(const GemmPlan& p, const CUtensorMap& tR, const CUtensorMap& tC, const GemmArgs& args,
+                       cudaStream_t s)
+{
+    auto kern = gemm_kernel<BM, BN, KIND, BLOCK, KPS>;
+    // the large dynamic shared-memory limit is a per-device function attribute
+    static bool configured[64] = {};
+    static std::mutex mu;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lk(mu);
+        if (!configured[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+            if (e != cudaSuccess) return e;
+            configured[dev] = true;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.G);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = p.smem_bytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (p.pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (p.cluster) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = (unsigned)p.split;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    return cudaLaunchKernelEx(&cfg, kern, tR, tC, args);
+}
+
+
+// Host accessor of this translation unit's device status word (defined once per unit
+// that includes this header).
+inline int status_word(int clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return W8_ERR_CUDA;
+    if (clear && v != 0) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return W8_ERR_CUDA;
+    }
+    return v;
+}
+
+struct GemmMaps {
+    CUtensorMap R, C;
+};
+
+// per-family launchers (one translation unit each)
+cudaError_t launch_f8(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_i8(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_block(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_bm64(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+int status_f8(int clear);
+int status_i8(int clear);
+int status_block(int clear);
+int status_bm64(int clear);
+
+}  // namespace gemm
+}  // namespace w8

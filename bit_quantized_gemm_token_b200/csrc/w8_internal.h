@@ -25,6 +25,10 @@ constexpr int kRowMaxK = 32768;   // longest row the register-resident row kerne
 // ---- GEMM (w8_gemm.cu) -------------------------------------------------------------------
 enum : int { kTileBN16 = 0, kTileBN32, kTileBN64, kTileBN128, kTileBN256, kNumTiles };
 
+// Split partitions keep one int32 ticket counter per output tile in the first
+// kMaxCounterTiles * 4 bytes of the workspace (256 KiB, the same for every shape).
+constexpr int kMaxCounterTiles = 65536;
+
 struct GemmPlan {
     int fmt;          // W8_FMT_*
     int M, N, K;
@@ -34,8 +38,12 @@ struct GemmPlan {
     int stream;       // balanced partition over the SMs
     int stages;
     int pdl;
+    int kps;          // 128-column K blocks per pipeline stage (1 or 2)
+    int cluster;      // split_k chunks run as one thread-block cluster per tile
+    int bm;           // rows of the MMA's M operand (128, or 64 for the narrow token tile)
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
+    int nsb;          // stage blocks (partition units) per tile
     long long units;
     int G;
     int align_tiles;

@@ -15,8 +15,9 @@
 // Layout of the work: the row kernels give one CTA per row and keep the row in
 // registers (16-byte vector loads, CPT chunks of 8 bf16 per thread); reductions are
 // warp shuffles plus one shared-memory stage.  The group kernel gives a half-warp per
-// 128-element group.  All kernels wait on the previous grid (programmatic dependent
-// launch) before reading and release their dependents right after.
+// 128-element group.  Under programmatic dependent launch every kernel releases its
+// dependents at entry (so the next GEMM can start streaming its weights) and waits for
+// the previous grid before it reads or writes anything.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -157,8 +158,8 @@ __global__ void __launch_bounds__(1024) quant_rows_kernel(const __nv_bfloat16* _
                                                           uint8_t* __restrict__ q, float* __restrict__ scale)
 {
     __shared__ float red[32];
+    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
     const int m = blockIdx.x;
     const int chunks = K >> 3;
     const __nv_bfloat16* xr = x + (size_t)m * ldx;
@@ -196,8 +197,8 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16
                                                              int ldx, uint8_t* __restrict__ q,
                                                              float* __restrict__ scale, int ue8m0)
 {
+    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
     const int gpr = K >> 7;
     const long long total = (long long)M * gpr;
     const long long gid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 4;
@@ -224,8 +225,8 @@ __global__ void __launch_bounds__(256) quant_weight_block_kernel(const __nv_bflo
                                                                  int ue8m0)
 {
     __shared__ float red[32];
+    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
     const int bk = blockIdx.x, bn = blockIdx.y;
     const int nbk = gridDim.x;
     const int rows = min(128, N - bn * 128), cols = min(128, K - bk * 128);
@@ -267,8 +268,8 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
 {
     __shared__ double redd[32];
     __shared__ float red[32];
+    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
     const int m = blockIdx.x;
     const int chunks = H >> 3;
     const __nv_bfloat16* xr = x + (size_t)m * ldx;
@@ -328,8 +329,8 @@ __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat1
                                                               uint8_t* __restrict__ q, float* __restrict__ scale)
 {
     __shared__ float red[32];
+    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
-    ptx::grid_dep_launch();
     const int m = blockIdx.x;
     const int chunks = I >> 3;
     const __nv_bfloat16* gr = xgu + (size_t)m * ld;

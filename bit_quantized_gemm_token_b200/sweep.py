@@ -1,0 +1,202 @@
+"""Offline variant sweep on the B200: for every (format, shape, M bucket) time the legal
+GEMM variants (Swap-AB / Standard, tile width, Standard / Split-K / balanced partition,
+K blocks per stage, CTAs per SM, pipeline depth) and write the fastest into the
+per-shape table that w8_load_table reads.  This is the role of the per-shape
+precomputed configs of the pages ("Helion nel backend vLLM ...", paragraphs 3-4), with
+an exhaustive search over a small space instead of their autotuner.
+
+Each candidate is checked before it is timed: its output must equal the reference
+variant's bit for bit for INT8 (int32 accumulators) and within the GEMM tolerance for
+the fp8 formats.  Timing: a CUDA graph of back-to-back launches (programmatic
+dependent launch, as in use) that rotate over enough weight copies to exceed 3x the
+L2, CUDA events on the capturing stream.
+
+    python -m bit_quantized_gemm_token_b200.sweep [--out PATH] [--quick] [--resume]
+"""
+import argparse
+import json
+import os
+import time
+
+import torch
+
+from . import w8
+
+DENSE = [(4096, 6144), (4096, 4096), (4096, 24576), (12288, 4096)]
+BLOCK = [(5120, 10240), (5120, 51200), (25600, 5120), (4096, 6144)]
+MS = [1, 2, 4, 8, 16, 32]
+HERE = os.path.dirname(os.path.abspath(__file__))
+DEFAULT_OUT = os.path.join(HERE, "tuning", "b200_table.txt")
+
+
+def candidates(fmt, M, N, K, quick=False):
+    block = fmt >= 2
+    out = []
+    bns = [b for b in (16, 32, 64) if b >= min(M, 64)][:2]
+    for bn in bns:
+        parts = [("stream", 1), ("stream", 2)] + [("split", s) for s in (1, 2, 4, 8, 16)] + \
+                [("cluster", s) for s in (2, 4, 8)]
+        for kind, arg in parts:
+            for kps in (1, 2):
+                for stages in ((0,) if quick else (0, 3, 4, 6)):
+                    if kind == "stream":
+                        v = w8.variant(True, 1, bn, stream=True, stages=stages, kps=kps, cps=arg)
+                    else:
+                        v = w8.variant(True, arg, bn, stages=stages, kps=kps, cluster=(kind == "cluster"))
+                    out.append(v)
+    if not block:
+        # Standard form, 64-row token tile, weights in the MMA's N slot
+        for bn in (128, 256):
+            parts = [("stream", 1), ("split", 1), ("split", 2), ("split", 4), ("split", 8), ("cluster", 2), ("cluster", 4)]
+            for kind, arg in parts:
+                for kps in (1, 2):
+                    for stages in ((0,) if quick else (0, 2, 3, 4)):
+                        if kind == "stream":
+                            v = w8.variant(False, 1, bn, stream=True, stages=stages, kps=kps, cps=arg, bm64=True)
+                        else:
+                            v = w8.variant(False, arg, bn, stages=stages, kps=kps, cluster=(kind == "cluster"), bm64=True)
+                        out.append(v)
+    legal = []
+    for v in out:
+        try:
+            w8.w8_gemm_resolve_variant(fmt, M, N, K, v)
+            legal.append(v)
+        except w8.W8Error:
+            pass
+    return sorted(set(legal))
+
+
+class Problem:
+    def __init__(self, fmt, N, K, ms, dev):
+        self.fmt, self.N, self.K = fmt, N, K
+        g = torch.Generator(device=dev)
+        g.manual_seed(4321 + N + K + fmt)
+        self.ncopy = max(2, -(-400_000_000 // (N * K)))
+        qf = w8.W8_Q_INT8 if fmt == 1 else w8.W8_Q_FP8
+        self.W = []
+        for _ in range(self.ncopy):
+            wb = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+            if fmt >= 2:
+                self.W.append(w8.w8_quant_weight_block(wb, ue8m0=(fmt == 3)))
+            else:
+                self.W.append(w8.w8_quant_per_token(wb, qf))
+            del wb
+        self.A = {}
+        for M in ms:
+            x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+            if fmt >= 2:
+                self.A[M] = w8.w8_quant_per_token(x, w8.W8_Q_FP8, group=128, ue8m0=(fmt == 3))
+            else:
+                self.A[M] = w8.w8_quant_per_token(x, qf)
+        self.ws = w8.Workspace(dev)
+        self.dev = dev
+
+    def run(self, M, v, copy=0, out=None):
+        A, sA = self.A[M]
+        Wq, sW = self.W[copy]
+        return w8.w8_gemm(self.fmt, A, sA, Wq, sW, out=out, variant=v, workspace=self.ws)
+
+    def check(self, M, v, ref_v):
+        A, _ = self.A[M]
+        if self.fmt == 1:
+            a = w8.w8_gemm_i32_debug(A, self.W[0][0], variant=v, workspace=self.ws)
+            b = w8.w8_gemm_i32_debug(A, self.W[0][0], variant=ref_v, workspace=self.ws)
+            torch.cuda.synchronize()
+            return torch.equal(a, b)
+        a = self.run(M, v).float()
+        b = self.run(M, ref_v).float()
+        torch.cuda.synchronize()
+        return bool(((a - b).abs().max() <= 2.0 ** -7 * b.abs().max() + 1e-3).item())
+
+    def time(self, M, v, reps=2):
+        out = torch.empty((M, self.N), dtype=torch.bfloat16, device=self.dev)
+        v = v | w8.W8_V_PDL
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        need = w8.w8_gemm_workspace_size(self.fmt, M, self.N, self.K, v)
+        self.ws.reserve(need)
+        with torch.cuda.stream(s):
+            self.run(M, v, 0, out)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for r in range(reps):
+                for c in range(self.ncopy):
+                    self.run(M, v, c, out)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        best = float("inf")
+        for _ in range(3):
+            with torch.cuda.stream(s):
+                e0.record(s)
+                g.replay()
+                e1.record(s)
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1) * 1e3 / (reps * self.ncopy))
+        del g
+        return best   # microseconds per launch
+
+
+def default_variant(fmt, M):
+    bn = 16 if M <= 16 else 32 if M <= 32 else 64
+    return w8.variant(True, 1, bn, stream=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--out", default=DEFAULT_OUT)
+    ap.add_argument("--quick", action="store_true", help="default pipeline depths only")
+    ap.add_argument("--formats", default="0,1,2")
+    ap.add_argument("--log", default="")
+    args = ap.parse_args()
+    os.environ["W8_TABLE"] = "none"
+    w8.w8_clear_table()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fmts = [int(f) for f in args.formats.split(",")]
+    rows = []
+    log = []
+    t_start = time.time()
+    for fmt in fmts:
+        shapes = BLOCK if fmt >= 2 else DENSE
+        for (K, N) in shapes:
+            prob = Problem(fmt, N, K, MS, dev)
+            for M in MS:
+                ref_v = default_variant(fmt, M)
+                res = []
+                for v in candidates(fmt, M, N, K, args.quick):
+                    if not prob.check(M, v, ref_v):
+                        log.append({"fmt": fmt, "N": N, "K": K, "M": M, "variant": hex(v), "error": "mismatch"})
+                        continue
+                    us = prob.time(M, v)
+                    res.append((us, v))
+                res.sort()
+                best_us, best_v = res[0]
+                base_us = [u for u, v in res if v == ref_v]
+                rec = {"fmt": fmt, "N": N, "K": K, "M": M, "best_us": round(best_us, 3), "variant": hex(best_v),
+                       "desc": w8.describe(best_v), "default_us": round(base_us[0], 3) if base_us else None,
+                       "TB/s": round((N * K + M * K + 2 * M * N) / (best_us * 1e-6) / 1e12, 3),
+                       "top5": [(round(u, 2), hex(v)) for u, v in res[:5]],
+                       "all": [(round(u, 2), hex(v)) for u, v in res]}
+                log.append(rec)
+                print(json.dumps({k: v for k, v in rec.items() if k != "all"}), flush=True)
+                for f in ([2, 3] if fmt == 2 else [fmt]):
+                    rows.append((f, N, K, M, best_v))
+            del prob
+            torch.cuda.empty_cache()
+    os.makedirs(os.path.dirname(args.out), exist_ok=True)
+    with open(args.out, "w") as fh:
+        fh.write("# per-shape GEMM variant table for B200 (sm_100a), written by\n")
+        fh.write("# python -m bit_quantized_gemm_token_b200.sweep; columns: fmt N K m_max variant\n")
+        fh.write("# fmt 0 = FP8-dynamic, 1 = W8A8-INT8, 2/3 = Block-FP8 (fp32 / UE8M0 scales)\n")
+        for r in rows:
+            fh.write("%d %d %d %d 0x%x\n" % r)
+    if args.log:
+        with open(args.log, "w") as fh:
+            json.dump(log, fh, indent=0)
+    print("wrote %d entries to %s in %.0f s" % (len(rows), args.out, time.time() - t_start))
+
+
+if __name__ == "__main__":
+    main()

@@ -13,6 +13,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libw8.so")
+DEFAULT_TABLE = os.path.join(_HERE, "tuning", "b200_table.txt")
 
 # status codes
 W8_OK = 0
@@ -36,11 +37,17 @@ W8_V_SPLIT_SHIFT = 4
 W8_V_TILE_SHIFT = 8
 W8_V_STAGES_SHIFT = 12
 W8_V_PDL = 1 << 16
+W8_V_CLUSTER = 1 << 17
+W8_V_BM64 = 1 << 18
+W8_V_KPS_SHIFT = 20
+W8_V_CPS_SHIFT = 22
 TILE_BN = {16: 0, 32: 1, 64: 2, 128: 3, 256: 4}
 
 
-def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stages: int = 0, pdl: bool = False) -> int:
-    """Explicit variant word (the W8_VARIANT macro plus stages / PDL bits)."""
+def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stages: int = 0, pdl: bool = False,
+            kps: int = 0, cps: int = 0, cluster: bool = False, bm64: bool = False) -> int:
+    """Explicit variant word (the W8_VARIANT macro plus stages, PDL, K blocks per stage
+    and CTAs per SM)."""
     lg = int(split).bit_length() - 1
     if split < 1 or (1 << lg) != split:
         raise ValueError("split must be a power of two")
@@ -48,8 +55,14 @@ def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stag
     v |= (lg & 0xF) << W8_V_SPLIT_SHIFT
     v |= (TILE_BN[bn] & 0xF) << W8_V_TILE_SHIFT
     v |= (stages & 0xF) << W8_V_STAGES_SHIFT
+    v |= (kps & 0x3) << W8_V_KPS_SHIFT
+    v |= (cps & 0x3) << W8_V_CPS_SHIFT
     if pdl:
         v |= W8_V_PDL
+    if cluster:
+        v |= W8_V_CLUSTER
+    if bm64:
+        v |= W8_V_BM64
     return v
 
 
@@ -57,7 +70,9 @@ def describe(v: int) -> dict:
     inv = {b: k for k, b in TILE_BN.items()}
     return {"swap_ab": bool(v & W8_V_SWAP_AB), "stream": bool(v & W8_V_STREAM),
             "split_k": 1 << ((v >> W8_V_SPLIT_SHIFT) & 0xF), "bn": inv.get((v >> W8_V_TILE_SHIFT) & 0xF),
-            "stages": (v >> W8_V_STAGES_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL)}
+            "stages": (v >> W8_V_STAGES_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL),
+            "kps": (v >> W8_V_KPS_SHIFT) & 0x3, "cps": (v >> W8_V_CPS_SHIFT) & 0x3,
+            "cluster": bool(v & W8_V_CLUSTER), "bm64": bool(v & W8_V_BM64)}
 
 
 class W8Error(RuntimeError):
@@ -98,6 +113,13 @@ def lib():
                "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
         getattr(L, fn).restype = I
     _lib = L
+    # the per-shape variant table shipped with the package (the offline sweep's output)
+    # is loaded once; W8_TABLE=<path> picks another one, W8_TABLE=none loads none
+    table = os.environ.get("W8_TABLE", DEFAULT_TABLE)
+    if table != "none" and os.path.exists(table):
+        n = L.w8_load_table(os.fsencode(table))
+        if n < 0:
+            raise W8Error("w8_load_table(%s)" % table, n)
     return L
 
 

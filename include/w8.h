@@ -83,7 +83,7 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 narrow slot over tokens (the Swap-AB variant, for small M);
  *                 otherwise the 128-row slot runs over tokens (Standard).
  *   split         log2 of split_k in bits 4..7 (split_k = 1..256, a power of two,
- *                 <= ceil(K/128)): every output tile's K range is cut into split_k
+ *                 <= the tile's stage blocks): every output tile's K range is cut into split_k
  *                 chunks, one CTA each, and the fp32 (int32 for INT8) partials are
  *                 added in a fixed order (Split-K).  split = 0 without W8_V_STREAM is
  *                 the Standard full-K tile loop.
@@ -93,10 +93,24 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 count); split bits are ignored.
  *   tile          bits 8..11, the narrow tile side BN: 0:16 1:32 2:64 3:128 4:256.
  *   stages        bits 12..15, shared-memory pipeline depth (0 = default).
- *   W8_V_PDL      launch with programmatic dependent launch: the kernel starts while
- *                 the previous kernel on the stream finishes and streams weight tiles
- *                 before waiting for it.  Only legal when W_q and the scales of W were
- *                 NOT written by the kernel launched immediately before this one.
+ *   W8_V_CLUSTER  Split-K whose split_k (2, 4 or 8) chunks of a tile run as one
+ *                 thread-block cluster: the partial accumulators are added in rank 0's
+ *                 shared memory through distributed shared memory (no workspace).
+ *   W8_V_BM64     Standard form with a 64-row token tile in the MMA's M slot and the
+ *                 weights in its N slot (tile 128 or 256; FP8 / INT8).  Each MMA then
+ *                 consumes BN weight rows; for decode sizes this carries twice the weight
+ *                 bytes per tensor-core instruction of the 128-row Swap-AB tile.
+ *   kps           bits 20..21, 128-column K blocks carried by one pipeline stage (0 =
+ *                 default: 2 for BN <= 64, else 1).  The partition unit is one stage
+ *                 block, so split_k must not exceed ceil(K / (128 * kps)).
+ *   ctas/SM       bits 22..23, CTAs per SM for W8_V_STREAM and the Standard loop
+ *                 (0 = 1).
+ *   W8_V_PDL      launch with programmatic dependent launch: the kernel may start while
+ *                 earlier kernels on the stream still run, and it reads weight tiles
+ *                 (into shared memory and L2) before waiting for them.  Only legal when
+ *                 W_q was not written by work still in flight on the stream -- the
+ *                 normal case of weights quantized once at load time.  Activations,
+ *                 scales, outputs and workspace are touched only after the wait.
  */
 #define W8_VARIANT_AUTO 0
 #define W8_V_EXPLICIT (1 << 0)
@@ -106,6 +120,10 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 #define W8_V_TILE_SHIFT 8
 #define W8_V_STAGES_SHIFT 12
 #define W8_V_PDL (1 << 16)
+#define W8_V_CLUSTER (1 << 17)
+#define W8_V_BM64 (1 << 18)
+#define W8_V_KPS_SHIFT 20
+#define W8_V_CPS_SHIFT 22
 #define W8_VARIANT(swap, log2_split, tile, stream)                                            \
     (W8_V_EXPLICIT | ((swap) ? W8_V_SWAP_AB : 0) | ((stream) ? W8_V_STREAM : 0) |            \
      (((log2_split) & 0xF) << W8_V_SPLIT_SHIFT) | (((tile) & 0xF) << W8_V_TILE_SHIFT))
@@ -166,10 +184,14 @@ W8_API int w8_silu_mul_quant(const void* gate_up, int M, int I, int ld, void* q,
  *   W_scale  fp32 [N] or [ceil(N/128), K/128] (BLOCK)
  *   out      bf16 [M, N], row-major
  *   workspace/ws_bytes  scratch for split partials and tile counters, sized by
- *            w8_gemm_workspace_size for the same (fmt, M, N, K, variant).  It must be
- *            zero-filled once before its first use; every successful call leaves its
- *            counter area zero again.  May be NULL when the size is 0.  Calls that
- *            share a workspace must not overlap on the device.
+ *            w8_gemm_workspace_size for the same (fmt, M, N, K, variant), 256-byte
+ *            aligned.  Its first 256 KiB hold per-tile counters (the same place for
+ *            every shape; at most 65536 output tiles per split call) and must be
+ *            zero-filled once before the first use; every successful call leaves them
+ *            zero again, so one workspace serves calls of any shape in sequence.  May
+ *            be NULL when the size is 0.  Calls that share a workspace must not run
+ *            concurrently on the device (successive launches on one stream are fine,
+ *            also with W8_V_PDL).  After W8_ERR_DEVICE_TIMEOUT, re-zero it.
  * Accuracy: max|out - ref| <= 2^-7 max|ref| + 1e-3 against the fp64 definition.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, NO_DEVICE, CUDA. */
 W8_API int w8_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale, void* out,

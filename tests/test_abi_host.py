@@ -69,6 +69,7 @@ def test_valid_call_without_device_reports_no_device(L):
 
 
 def test_variant_resolution_and_workspace(L):
+    w8.w8_clear_table()   # the built-in rule, not the shipped table
     # decode: Swap-AB with the narrow token tile, balanced partition
     v = w8.w8_gemm_resolve_variant(0, 1, 4096, 4096)
     d = w8.describe(v)
@@ -84,8 +85,8 @@ def test_variant_resolution_and_workspace(L):
     # workspace: none for whole-tile partitions, some for split / balanced
     assert w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=1, bn=16)) == 0
     n = w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=4, bn=16))
-    tiles = 2
-    assert n == 256 + tiles * 4 * 2 * 16 * 128 * 4
+    ctas = 2 * 4                                  # 2 tiles x split 4
+    assert n == 65536 * 4 + ctas * 2 * 16 * 128 * 4
     assert w8.w8_gemm_workspace_size(0, 8, 4096, 4096, 0) > 0
 
 
@@ -107,3 +108,5 @@ def test_table_parsing(L, tmp_path):
     finally:
         w8.w8_clear_table()
     assert w8.w8_gemm_resolve_variant(0, 8, 4096, 4096) != v1
+    if os.path.exists(w8.DEFAULT_TABLE):
+        assert w8.w8_load_table(w8.DEFAULT_TABLE) > 0

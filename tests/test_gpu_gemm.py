@@ -25,10 +25,18 @@ VARIANTS = {
     "std256_stream": w8.variant(False, 1, 256, stream=True),
     "std32_split8": w8.variant(False, 8, 32),
     "swap16_pdl": w8.variant(True, 1, 16, stream=True, pdl=True),
+    "swap16_cluster4": w8.variant(True, 4, 16, cluster=True),
+    "swap32_cluster2_kps1": w8.variant(True, 2, 32, cluster=True, kps=1),
+    "swap16_cluster8_pdl": w8.variant(True, 8, 16, cluster=True, kps=1, pdl=True),
+    "std128_cluster2": w8.variant(False, 2, 128, cluster=True),
+    "bm64_256_stream": w8.variant(False, 1, 256, stream=True, bm64=True),
+    "bm64_128_split2_kps2": w8.variant(False, 2, 128, bm64=True, kps=2, stages=2),
+    "bm64_256_cluster2": w8.variant(False, 2, 256, cluster=True, bm64=True, stages=3),
+    "bm64_256_split4_pdl": w8.variant(False, 4, 256, bm64=True, stages=2, pdl=True),
 }
 
 BLOCK_OK = {"auto", "swap16", "swap32_split2", "swap16_stream", "swap64_split4", "std64_split4", "std32_split8",
-            "swap16_pdl"}
+            "swap16_pdl", "swap16_cluster4", "swap32_cluster2_kps1", "swap16_cluster8_pdl"}
 
 _cache = {}
 
@@ -168,3 +176,17 @@ def test_graph_capture_small_m(orc):
     torch.cuda.synchronize()
     assert torch.equal(out, eager)
     assert_bf16_close(out, ref, "graph")
+
+
+def test_workspace_shared_across_shapes(orc):
+    """One workspace for calls of different shapes in sequence: the partial sums of a
+    call with few tiles must not be read as ticket counters by a call with many."""
+    ws = w8.Workspace()
+    for (M, N, K, v) in [(16, 256, 4096, w8.variant(True, 32, 16)), (1, 8192, 1024, w8.variant(True, 1, 16, stream=True)),
+                         (3, 512, 2048, w8.variant(True, 16, 16)), (1, 8192, 1024, w8.variant(True, 1, 16, stream=True))]:
+        Aq, sA, Wq, sW, ref, _ = operands(orc, 0, M, N, K)
+        out = poison_bf16((M, N))
+        w8.w8_gemm(0, dev_codes(Aq, 0), dev_f32(sA), dev_codes(Wq, 0), dev_f32(sW), out=out, variant=v, workspace=ws)
+        torch.cuda.synchronize()
+        assert_bf16_close(out, ref, "shared workspace %s" % ((M, N, K),))
+    assert int(ws.buf[:65536 * 4].sum()) == 0
