@@ -212,6 +212,23 @@ W8_API int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant);
 W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int N, int K, int variant,
                       void* workspace, size_t ws_bytes, w8_stream_t stream);
 
+/* w8_gemm for callers that cannot allocate device memory.  (An addition of this
+ * library: the pages describe no counterpart.)  Some callers cannot provide the
+ * Split-K workspace because they may not call cudaMalloc -- code running inside a
+ * runtime whose allocator it does not own, or a service whose device memory is fixed
+ * at start-up.  This entry point takes the same arguments as w8_gemm minus the
+ * workspace and uses instead a scratch array the library places in device memory when
+ * it is loaded: 8 MiB per GPU, held until the process exits.  A variant whose
+ * workspace would exceed that (see w8_gemm_workspace_size) returns W8_ERR_WORKSPACE.
+ * It allocates nothing: the first call on each device looks up the array's device
+ * address (a runtime query, no allocation); make that first call before any stream
+ * capture.  Each call clears the ticket counters it uses with cudaMemsetAsync on
+ * `stream`.  All calls on a device share the array, so calls that overlap on the GPU
+ * (e.g. on two streams at once) race; successive calls on one stream are fine.
+ * Errors: as w8_gemm. */
+W8_API int w8_gemm_noalloc(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
+                           void* out, int M, int N, int K, int variant, w8_stream_t stream);
+
 /* Per-shape variant table (the output of the offline sweep).  Text, one entry per line:
  *   <fmt> <N> <K> <m_max> <variant as 0x hex>
  * '#' starts a comment.  AUTO picks the entry with the same (fmt, N, K) and the
