@@ -42,10 +42,9 @@ constexpr int tile_bn(int id) { return 16 << id; }
 
 size_t stage_bytes(int bm, int bn, int kps) { return (size_t)kps * ((size_t)bm * 128 + (size_t)bn * 128); }
 
-size_t smem_for(int bm, int bn, int kps, int stages, int csplit)
+size_t smem_for(int bm, int bn, int kps, int stages)
 {
-    const size_t red = csplit > 1 ? (size_t)(csplit - 1) * bn * bm * 4 : 0;
-    return 1024 + (size_t)stages * stage_bytes(bm, bn, kps) + (size_t)(2 * stages + 2 * kNumAcc + 2) * 8 + 16 + red;
+    return 1024 + (size_t)stages * stage_bytes(bm, bn, kps) + (size_t)(2 * stages + 2 * kNumAcc + 3) * 8 + 16;
 }
 
 int default_stages(int bn, int kps)
@@ -109,7 +108,10 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
     if (stages == 0) stages = default_stages(q.bn, kps);
     if (stages < 2) return W8_ERR_UNSUPPORTED;
     q.stages = stages;
-    q.smem_bytes = smem_for(q.bm, q.bn, kps, stages, q.cluster ? (1 << lg) : 0);
+    q.smem_bytes = smem_for(q.bm, q.bn, kps, stages);
+    // the cluster reduction reuses rank 0's stage memory for the other ranks' partials
+    if (q.cluster && (size_t)((1 << lg) - 1) * q.bn * q.bm * 4 > (size_t)stages * stage_bytes(q.bm, q.bn, kps))
+        return W8_ERR_UNSUPPORTED;
     if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
     if (cps == 0) cps = 1;
 

@@ -236,12 +236,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + kNumAcc;
     uint64_t* drain = tempty + kNumAcc;
-    uint64_t* red_full = drain + 1;   // cluster split: partials of the other ranks have landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_full + 1);
+    uint64_t* red_full = drain + 1;   // cluster split (rank 0): partials of the other ranks have landed
+    uint64_t* red_go = red_full + 1;  // cluster split (ranks 1..): rank 0's stage memory is free
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_go + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* ticket = reinterpret_cast<volatile int*>(tmem_slot + 2);
-    // cluster split: [csplit - 1][BN columns][128 rows] partial words, used in rank 0 only
-    uint32_t* red_buf = reinterpret_cast<uint32_t*>(tmem_slot + 4);
+    // cluster split: [csplit - 1][BN columns][BM rows] partial words, written into rank 0's
+    // stage memory once its last MMA has completed (the stages are free by then)
+    uint32_t* red_buf = reinterpret_cast<uint32_t*>(smem);
     // stage s: R slots [KPS][128 x 128 B], then C slots [KPS][BN x 128 B]; all 1024-aligned
     auto r_slot = [&](int s, int j) { return smem + (size_t)s * kStageBytes + (size_t)j * kRBytes; };
     auto c_slot = [&](int s, int j) { return smem + (size_t)s * kStageBytes + (size_t)KPS * kRBytes + (size_t)j * kCBytes; };
@@ -259,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::mbar_init(ptx::smem_u32(drain), 1);
         ptx::mbar_init(ptx::smem_u32(red_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * kEpiThreads : 1u);
+        ptx::mbar_init(ptx::smem_u32(red_go), 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -520,9 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (a.csplit > 1) {
                 // ---- cluster split: ranks 1.. write their partial accumulators into rank
                 // 0's shared memory (distributed shared memory) and arrive on its barrier;
-                // rank 0 adds them in rank order, scales and stores
+                // rank 0 adds them in rank order, scales and stores.  The partials land in
+                // rank 0's stage memory, so rank 0 first tells the others (remote arrive
+                // on their `red_go`) that its MMAs -- the last readers of that memory --
+                // have completed, which its accumulator being ready implies.
                 const uint32_t rank = ptx::cluster_ctarank();
                 if (rank != 0) {
+                    const bool g = wait_bounded<true>(ptx::smem_u32(red_go), 0, abort_flag);
+                    if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !g)) { ok = false; break; }
                     const uint32_t rbase = ptx::map_to_rank(ptx::smem_u32(red_buf), 0) +
                                            (rank - 1) * (uint32_t)(BN * BM * 4);
 #pragma unroll
@@ -536,6 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(red_full), 0));
                 } else {
+                    if (first_epi)
+                        for (int r = 1; r < a.csplit; ++r) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(red_go), (uint32_t)r));
                     const bool w = wait_bounded<true>(ptx::smem_u32(red_full), 0, abort_flag);
                     if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) { ok = false; break; }
 #pragma unroll
