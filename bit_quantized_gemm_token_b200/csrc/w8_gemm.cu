@@ -109,9 +109,13 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
     if (stages < 2) return W8_ERR_UNSUPPORTED;
     q.stages = stages;
     q.smem_bytes = smem_for(q.bm, q.bn, kps, stages);
-    // the cluster reduction reuses rank 0's stage memory for the other ranks' partials
-    if (q.cluster && (size_t)((1 << lg) - 1) * q.bn * q.bm * 4 > (size_t)stages * stage_bytes(q.bm, q.bn, kps))
-        return W8_ERR_UNSUPPORTED;
+    // the cluster reduction reuses rank 0's stage memory for the partials: the other
+    // ranks' [BN][BM] tiles, or, with the 64-row token tile, every rank's real rows
+    if (q.cluster) {
+        const size_t red = (q.bm == 64) ? (size_t)(1 << lg) * (size_t)(M < 64 ? M : 64) * q.bn * 4
+                                        : (size_t)((1 << lg) - 1) * q.bn * q.bm * 4;
+        if (red > (size_t)stages * stage_bytes(q.bm, q.bn, kps)) return W8_ERR_UNSUPPORTED;
+    }
     if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
     if (cps == 0) cps = 1;
 

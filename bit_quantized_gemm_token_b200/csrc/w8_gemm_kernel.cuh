@@ -52,7 +52,7 @@ constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiBarrier = 1;          // named barrier id of the epilogue warps
 constexpr int kTmemBarrier = 2;         // named barrier id of warps 1..5 (TMEM hand-off)
-constexpr int kNumAcc = 2;              // TMEM accumulator buffers
+constexpr int kNumAcc = 2;              // TMEM accumulator barrier slots (buffers in use: kAccBufs)
 constexpr unsigned long long kWaitNs = 1000000000ull;   // 1 s bound on any single wait
 constexpr int kL2Ahead = 6;             // units whose weights are prefetched to L2 before the PDL wait
 
@@ -225,7 +225,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kRBytes = BM * 128;
     constexpr int kCBytes = BN * 128;
     constexpr int kStageBytes = KPS * (kRBytes + kCBytes);
-    constexpr uint32_t kTmemCols = (kNumAcc * BN <= 32) ? 32 : (kNumAcc * BN <= 64) ? 64 : (kNumAcc * BN <= 128) ? 128 : (kNumAcc * BN <= 256) ? 256 : 512;
+    // accumulators in TMEM: double-buffered, except for the 64-row token tile, whose single
+    // 256-column buffer leaves room for a CTA of the next kernel on the same SM
+    constexpr int kAccBufs = (BM == 64) ? 1 : 2;
+    constexpr uint32_t kTmemCols = (kAccBufs * BN <= 32) ? 32 : (kAccBufs * BN <= 64) ? 64 : (kAccBufs * BN <= 128) ? 128 : (kAccBufs * BN <= 256) ? 256 : 512;
     constexpr uint32_t kIdesc = instr_desc<KIND, BM, BN>();
 
     extern __shared__ uint8_t smem_raw[];
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (BLOCK) {
                             ptx::mma_commit(ptx::smem_u32(tfull + b));
-                            if (++b == kNumAcc) { b = 0; bp ^= 1u; }
+                            if (++b == kAccBufs) { b = 0; bp ^= 1u; }
                             ++nbuf_used;
                         }
                     }
@@ -400,9 +403,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++stage == S) { stage = 0; phase ^= 1u; }
             if (BLOCK) {
                 for (int j = 0; j < nbuf_used; ++j)
-                    if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+                    if (++buf == kAccBufs) { buf = 0; bphase ^= 1u; }
             } else if (seg_last) {
-                if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+                if (++buf == kAccBufs) { buf = 0; bphase ^= 1u; }
             }
         }
         if (!ok && lane == 0) {
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(tempty + buf));
-                    if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+                    if (++buf == kAccBufs) { buf = 0; bphase ^= 1u; }
                 }
                 if (!ok) break;
             } else {
@@ -520,7 +523,78 @@ __global__ void __launch_bounds__(kThreads, 1)
             // columns of this tile that hold real rows of the C operand (tokens for
             // Swap-AB: only these are written, published and reduced)
             const int ncv = (a.rows_C - ct * BN < BN) ? a.rows_C - ct * BN : BN;
-            if (a.csplit > 1) {
+            // 64-row token tile: only nrows rows are real tokens; its partials are kept as
+            // [row][column] and reduced column-parallel by all 128 epilogue threads
+            constexpr bool kCompact = (BM == 64);
+            const int nrows = (a.rows_R - rt * BM < BM) ? a.rows_R - rt * BM : BM;
+            const int te = threadIdx.x - 64;   // epilogue thread index 0..127
+            // publish this thread's row (if any) as BN contiguous words at dst (generic or
+            // cluster-shared address space)
+            auto publish_row = [&](uint32_t* gdst, uint32_t sdst, bool remote) {
+#pragma unroll
+                for (int c0 = 0; c0 < BN; c0 += 16) {
+                    if (c0 >= ncv) break;
+                    uint32_t v[16];
+                    fetch16(c0, v);
+                    if (has_row) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            if (remote) {
+                                ptx::st_cluster_v4(sdst + (uint32_t)((c0 + 4 * q4) * 4), v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                            } else {
+                                uint4 w4 = make_uint4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                                __stcg(reinterpret_cast<uint4*>(gdst + c0 + 4 * q4), w4);
+                            }
+                        }
+                    }
+                }
+            };
+            // finish output column `col` of row r from a summed word
+            auto finish = [&](int r, int col, uint32_t w) {
+                const int m = rt * BM + r;
+                const float sr = (a.out_i32 == nullptr) ? __ldg(a.sA + m) : 1.0f;
+                store_out<KIND, BLOCK>(a, m, ct * BN + col, w, sr);
+            };
+            if (kCompact && a.csplit > 1) {
+                // ---- cluster split, 64-row token tile: every rank's real rows go to rank 0's
+                // stage memory as [rank][row][column]; rank 0 sums ranks in order per column
+                const uint32_t rank = ptx::cluster_ctarank();
+                const uint32_t slot_words = (uint32_t)(nrows * BN);
+                if (rank != 0) {
+                    const bool g = wait_bounded<true>(ptx::smem_u32(red_go), 0, abort_flag);
+                    if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !g)) { ok = false; break; }
+                    const uint32_t rbase = ptx::map_to_rank(ptx::smem_u32(red_buf), 0) +
+                                           (rank * slot_words + (uint32_t)(i * BN)) * 4;
+                    publish_row(nullptr, rbase, true);
+                    ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(red_full), 0));
+                } else {
+                    if (first_epi)
+                        for (int r = 1; r < a.csplit; ++r) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(red_go), (uint32_t)r));
+#pragma unroll
+                    for (int c0 = 0; c0 < BN; c0 += 16) {
+                        if (c0 >= ncv) break;
+                        uint32_t v[16];
+                        fetch16(c0, v);
+                        if (has_row)
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) red_buf[i * BN + c0 + jj] = v[jj];
+                    }
+                    ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                    const bool w = wait_bounded<true>(ptx::smem_u32(red_full), 0, abort_flag);
+                    if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) { ok = false; break; }
+                    for (int col = te; col < ncv; col += kEpiThreads)
+                        for (int r = 0; r < nrows; ++r) {
+                            uint32_t v = red_buf[r * BN + col];
+                            for (int k = 1; k < a.csplit; ++k)
+                                v = add_words<KIND>(v, red_buf[k * slot_words + r * BN + col]);
+                            finish(r, col, v);
+                        }
+                }
+            } else if (kCompact && !full_tile) {
+                // ---- partial, 64-row token tile: [row][column] words, one row per thread
+                uint32_t* my = a.partials + ((size_t)blockIdx.x * 2 + slot) * (size_t)(BN * BM);
+                publish_row(my + (size_t)(has_row ? i : 0) * BN, 0u, false);
+            } else if (a.csplit > 1) {
                 // ---- cluster split: ranks 1.. write their partial accumulators into rank
                 // 0's shared memory (distributed shared memory) and arrive on its barrier;
                 // rank 0 adds them in rank order, scales and stores.  The partials land in
@@ -588,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(tempty + buf));
-                if (++buf == kNumAcc) { buf = 0; bphase ^= 1u; }
+                if (++buf == kAccBufs) { buf = 0; bphase ^= 1u; }
             }
             if (!full_tile && a.csplit <= 1) {
                 // ---- ticket: the last contributor of tile t finishes it
@@ -598,7 +672,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
                 const int g_lo = cta_of_unit(a, (long long)t * nsb);
                 const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1);
-                if (*ticket == g_hi - g_lo) {
+                if (*ticket == g_hi - g_lo && kCompact) {
+                    // column-parallel: per column and row, contributors added in CTA order,
+                    // four contributors' loads in flight together
+                    __threadfence();
+                    const int nc = g_hi - g_lo + 1;
+                    for (int col = te; col < ncv; col += kEpiThreads)
+                        for (int r0 = 0; r0 < nrows; r0 += 8) {
+                            // 8 rows x 4 contributors of loads in flight per round trip
+                            uint32_t v[8];
+#pragma unroll
+                            for (int rr = 0; rr < 8; ++rr) v[rr] = 0u;
+                            for (int cb = 0; cb < nc; cb += 4) {
+                                uint32_t x[4][8];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const int c = g_lo + cb + k;
+                                    const uint32_t* p = nullptr;
+                                    if (cb + k < nc) {
+                                        const int sl = (unit_begin(a, c) / nsb == t) ? 0 : 1;
+                                        p = a.partials + ((size_t)c * 2 + sl) * (size_t)(BN * BM) + col;
+                                    }
+#pragma unroll
+                                    for (int rr = 0; rr < 8; ++rr)
+                                        x[k][rr] = (p != nullptr && r0 + rr < nrows) ? __ldcg(p + (size_t)(r0 + rr) * BN) : 0u;
+                                }
+#pragma unroll
+                                for (int k = 0; k < 4; ++k)
+                                    if (cb + k < nc)
+#pragma unroll
+                                        for (int rr = 0; rr < 8; ++rr)
+                                            v[rr] = (cb + k == 0) ? x[k][rr] : add_words<KIND>(v[rr], x[k][rr]);
+                            }
+#pragma unroll
+                            for (int rr = 0; rr < 8; ++rr)
+                                if (r0 + rr < nrows) finish(r0 + rr, col, v[rr]);
+                        }
+                    if (first_epi) a.counters[t] = 0;   // leave the counter ready for the next call
+                } else if (*ticket == g_hi - g_lo) {
                     __threadfence();
                     const int nc = g_hi - g_lo + 1;
 #pragma unroll 1

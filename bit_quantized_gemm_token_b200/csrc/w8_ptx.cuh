@@ -126,6 +126,12 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v)
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
 // Arrive (release, cluster scope) on an mbarrier in another CTA of the cluster: this
 // thread's earlier shared::cluster stores are visible to whoever acquires the phase.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar)

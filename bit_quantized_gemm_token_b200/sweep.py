@@ -7,9 +7,9 @@ an exhaustive search over a small space instead of their autotuner.
 
 Each candidate is checked before it is timed: its output must equal the reference
 variant's bit for bit for INT8 (int32 accumulators) and within the GEMM tolerance for
-the fp8 formats.  Timing: a CUDA graph of back-to-back launches (programmatic
-dependent launch, as in use) that rotate over enough weight copies to exceed 3x the
-L2, CUDA events on the capturing stream.
+the fp8 formats.  Timing: a CUDA graph of (activation quant, GEMM) pairs, as in use,
+with programmatic dependent launch, rotating over enough weight copies to exceed 3x
+the L2; CUDA events on the capturing stream; the time per pair is reported.
 
     python -m bit_quantized_gemm_token_b200.sweep [--out PATH] [--quick] [--resume]
 """
@@ -81,15 +81,21 @@ class Problem:
             else:
                 self.W.append(w8.w8_quant_per_token(wb, qf))
             del wb
-        self.A = {}
+        self.A, self.X = {}, {}
+        self.qf = qf
         for M in ms:
             x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
-            if fmt >= 2:
-                self.A[M] = w8.w8_quant_per_token(x, w8.W8_Q_FP8, group=128, ue8m0=(fmt == 3))
-            else:
-                self.A[M] = w8.w8_quant_per_token(x, qf)
+            self.X[M] = x
+            self.A[M] = self.quant(M)
         self.ws = w8.Workspace(dev)
         self.dev = dev
+
+    def quant(self, M):
+        A = self.A.get(M)
+        q, s = (A if A is not None else (None, None))
+        if self.fmt >= 2:
+            return w8.w8_quant_per_token(self.X[M], w8.W8_Q_FP8, group=128, ue8m0=(self.fmt == 3), q=q, scale=s)
+        return w8.w8_quant_per_token(self.X[M], self.qf, q=q, scale=s)
 
     def run(self, M, v, copy=0, out=None):
         A, sA = self.A[M]
@@ -122,6 +128,8 @@ class Problem:
         with torch.cuda.graph(g, stream=s):
             for r in range(reps):
                 for c in range(self.ncopy):
+                    # as in use: the activation quantizer runs right before every GEMM
+                    self.quant(M)
                     self.run(M, v, c, out)
         g.replay()
         torch.cuda.synchronize()

@@ -12,7 +12,7 @@ from gpu_helpers import assert_bf16_close, dev_codes, dev_f32, poison_bf16, quan
 pytestmark = pytest.mark.gpu
 
 SHAPES = [(1, 256, 256), (5, 384, 1024), (16, 300, 640), (17, 1000, 1040), (32, 2048, 1024),
-          (33, 256, 512), (100, 520, 768), (130, 1024, 2048)]
+          (33, 256, 512), (64, 1024, 2048), (100, 520, 768), (130, 1024, 2048)]
 
 VARIANTS = {
     "auto": w8.W8_VARIANT_AUTO,
@@ -33,6 +33,8 @@ VARIANTS = {
     "bm64_128_split2_kps2": w8.variant(False, 2, 128, bm64=True, kps=2, stages=2),
     "bm64_256_cluster2": w8.variant(False, 2, 256, cluster=True, bm64=True, stages=3),
     "bm64_256_split4_pdl": w8.variant(False, 4, 256, bm64=True, stages=2, pdl=True),
+    "bm64_256_cluster4": w8.variant(False, 4, 256, cluster=True, bm64=True, stages=3),
+    "bm64_128_stream2": w8.variant(False, 1, 128, stream=True, bm64=True, cps=2, stages=2),
 }
 
 BLOCK_OK = {"auto", "swap16", "swap32_split2", "swap16_stream", "swap64_split4", "std64_split4", "std32_split8",
