@@ -157,7 +157,21 @@ int w8_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, 
     if (H > kRowMaxK) return W8_ERR_UNSUPPORTED;
     int rc = check_device(nullptr);
     if (rc != W8_OK) return rc;
-    return launch_rmsnorm_quant(x, gamma, eps, M, H, ldx, q, scale, reinterpret_cast<cudaStream_t>(stream));
+    return launch_rmsnorm_quant(x, gamma, eps, M, H, ldx, q, scale, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_rmsnorm_quant_group(const void* x, const void* gamma, float eps, int M, int H, int ldx, int group, int ue8m0,
+                           void* q, float* scale, w8_stream_t stream)
+{
+    if (!row_args_ok(x, M, H, ldx, q, scale) || !gamma) return W8_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f)) return W8_ERR_INVALID_ARG;
+    if (group != 128 || H % group != 0) return W8_ERR_UNSUPPORTED;
+    if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(gamma, 16) || !aligned(q, 8) || !aligned(scale, 4))
+        return W8_ERR_ALIGNMENT;
+    if (H > kRowMaxK) return W8_ERR_UNSUPPORTED;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    return launch_rmsnorm_quant(x, gamma, eps, M, H, ldx, q, scale, group, ue8m0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8_silu_mul_quant(const void* gate_up, int M, int I, int ld, void* q, float* scale, w8_stream_t stream)
@@ -168,7 +182,19 @@ int w8_silu_mul_quant(const void* gate_up, int M, int I, int ld, void* q, float*
     if (I > kRowMaxK) return W8_ERR_UNSUPPORTED;
     int rc = check_device(nullptr);
     if (rc != W8_OK) return rc;
-    return launch_silu_mul_quant(gate_up, M, I, ld, q, scale, reinterpret_cast<cudaStream_t>(stream));
+    return launch_silu_mul_quant(gate_up, M, I, ld, q, scale, 0, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_silu_mul_quant_group(const void* gate_up, int M, int I, int ld, int group, int ue8m0, void* q, float* scale,
+                            w8_stream_t stream)
+{
+    if (!gate_up || !q || !scale || M <= 0 || I <= 0 || ld < 2 * I) return W8_ERR_INVALID_ARG;
+    if (group != 128 || I % group != 0) return W8_ERR_UNSUPPORTED;
+    if (ld % 8 != 0 || !aligned(gate_up, 16) || !aligned(q, 8) || !aligned(scale, 4)) return W8_ERR_ALIGNMENT;
+    if (I > kRowMaxK) return W8_ERR_UNSUPPORTED;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    return launch_silu_mul_quant(gate_up, M, I, ld, q, scale, group, ue8m0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int w8_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale, void* out, int M,

@@ -17,8 +17,9 @@ int launch_quant_rows(int qfmt, const void* x, int M, int K, int ldx, void* q, f
 int launch_quant_group128(const void* x, int M, int K, int ldx, void* q, float* scale, int ue8m0, cudaStream_t s);
 int launch_quant_weight_block(const void* w, int N, int K, void* q, float* scale, int ue8m0, cudaStream_t s);
 int launch_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, int ldx, void* q, float* scale,
-                         cudaStream_t s);
-int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float* scale, cudaStream_t s);
+                         int group, int ue8m0, cudaStream_t s);
+int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float* scale, int group, int ue8m0,
+                          cudaStream_t s);
 
 constexpr int kRowMaxK = 32768;   // longest row the register-resident row kernels accept
 

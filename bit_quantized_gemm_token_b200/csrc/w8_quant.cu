@@ -152,6 +152,25 @@ __device__ __forceinline__ float exp_cw(float x)
     return __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
 }
 
+// Grouped (1x128) variant of the last step of the row kernels: the 16 chunks of a
+// 128-element group sit in 16 consecutive lanes (chunk index = thread + c * blockDim,
+// blockDim a multiple of 32), so the group's amax is a half-warp reduction.  Writes the
+// chunk's 8 codes and, from the group's first lane, its scale.
+__device__ __forceinline__ void encode_chunk_grouped(const float (&y)[8], int idx, int ng, bool ue8m0,
+                                                     uint8_t* qrow, float* srow)
+{
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
+    const unsigned hmask = 0xFFFFu << (threadIdx.x & 16);
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
+    const float s = scale_from_amax(amax, kE4M3Max, ue8m0);
+    if ((idx & 15) == 0) srow[idx >> 4] = s;
+    (void)ng;
+    *reinterpret_cast<uint2*>(qrow + (size_t)idx * 8) = encode8<W8_Q_FP8>(y, s);
+}
+
 // ------------------------------------------------------------------- per-token rows
 template <int QFMT, int CPT>
 __global__ void __launch_bounds__(1024) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int K, int ldx,
@@ -260,11 +279,11 @@ __global__ void __launch_bounds__(256) quant_weight_block_kernel(const __nv_bflo
 }
 
 // ------------------------------------------------------------------- rms_norm + quant
-template <int CPT>
+template <int CPT, bool GROUPED>
 __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16* __restrict__ x,
                                                              const __nv_bfloat16* __restrict__ gamma, float eps,
                                                              int H, int ldx, uint8_t* __restrict__ q,
-                                                             float* __restrict__ scale)
+                                                             float* __restrict__ scale, int ue8m0)
 {
     __shared__ double redd[32];
     __shared__ float red[32];
@@ -292,6 +311,23 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
     ss = block_sum_f64(ss, redd);
     const float mean = __fdiv_rn(__double2float_rn(ss), (float)H);
     const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+    if (GROUPED) {
+        // rms_norm_per_block_quant: y = (x * r) * gamma, then one scale per 1x128 group
+        const int ng = H >> 7;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int idx = threadIdx.x + c * blockDim.x;
+            if (idx < chunks) {
+                float f[8], g[8], y[8];
+                unpack_bf16x8(raw[c], f);
+                unpack_bf16x8(ld_nc_v4(gamma + (size_t)idx * 8), g);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(f[i], r), g[i]);
+                encode_chunk_grouped(y, idx, ng, ue8m0 != 0, q + (size_t)m * H, scale + (size_t)m * ng);
+            }
+        }
+        return;
+    }
     // y = (x * r) * gamma, recomputed in the second pass rather than kept
     float amax = 0.0f;
 #pragma unroll
@@ -324,9 +360,10 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
 }
 
 // ------------------------------------------------------------------- silu_and_mul + quant
-template <int CPT>
+template <int CPT, bool GROUPED>
 __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat16* __restrict__ xgu, int I, int ld,
-                                                              uint8_t* __restrict__ q, float* __restrict__ scale)
+                                                              uint8_t* __restrict__ q, float* __restrict__ scale,
+                                                              int ue8m0)
 {
     __shared__ float red[32];
     ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
@@ -351,6 +388,16 @@ __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat1
                 amax = fmaxf(amax, fabsf(h[c][i]));
             }
         }
+    }
+    if (GROUPED) {
+        // silu_and_mul_per_block_quant: one scale per 1x128 group of h
+        const int ng = I >> 7;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int idx = threadIdx.x + c * blockDim.x;
+            if (idx < chunks) encode_chunk_grouped(h[c], idx, ng, ue8m0 != 0, q + (size_t)m * I, scale + (size_t)m * ng);
+        }
+        return;
     }
     amax = block_max(amax, red);
     const float s = scale_from_amax(amax, kE4M3Max, false);
@@ -438,28 +485,39 @@ int launch_quant_weight_block(const void* w, int N, int K, void* q, float* scale
 }
 
 int launch_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int H, int ldx, void* q, float* scale,
-                         cudaStream_t s)
+                         int group, int ue8m0, cudaStream_t s)
 {
     int threads, cpt;
     if (!row_shape(H / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
     const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(gamma);
     uint8_t* qp = static_cast<uint8_t*>(q);
-    void* args[] = {(void*)&xp, (void*)&gp, (void*)&eps, (void*)&H, (void*)&ldx, (void*)&qp, (void*)&scale};
-    const void* fn = cpt == 1 ? (const void*)rmsnorm_quant_kernel<1>
-                              : cpt == 2 ? (const void*)rmsnorm_quant_kernel<2> : (const void*)rmsnorm_quant_kernel<4>;
+    void* args[] = {(void*)&xp, (void*)&gp, (void*)&eps, (void*)&H, (void*)&ldx, (void*)&qp, (void*)&scale, (void*)&ue8m0};
+    const void* fn;
+    if (group)
+        fn = cpt == 1 ? (const void*)rmsnorm_quant_kernel<1, true>
+                      : cpt == 2 ? (const void*)rmsnorm_quant_kernel<2, true> : (const void*)rmsnorm_quant_kernel<4, true>;
+    else
+        fn = cpt == 1 ? (const void*)rmsnorm_quant_kernel<1, false>
+                      : cpt == 2 ? (const void*)rmsnorm_quant_kernel<2, false> : (const void*)rmsnorm_quant_kernel<4, false>;
     return status_of(launch(fn, dim3(M), dim3(threads), args, s));
 }
 
-int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float* scale, cudaStream_t s)
+int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float* scale, int group, int ue8m0,
+                          cudaStream_t s)
 {
     int threads, cpt;
     if (!row_shape(I / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(xgu);
     uint8_t* qp = static_cast<uint8_t*>(q);
-    void* args[] = {(void*)&xp, (void*)&I, (void*)&ld, (void*)&qp, (void*)&scale};
-    const void* fn = cpt == 1 ? (const void*)silu_mul_quant_kernel<1>
-                              : cpt == 2 ? (const void*)silu_mul_quant_kernel<2> : (const void*)silu_mul_quant_kernel<4>;
+    void* args[] = {(void*)&xp, (void*)&I, (void*)&ld, (void*)&qp, (void*)&scale, (void*)&ue8m0};
+    const void* fn;
+    if (group)
+        fn = cpt == 1 ? (const void*)silu_mul_quant_kernel<1, true>
+                      : cpt == 2 ? (const void*)silu_mul_quant_kernel<2, true> : (const void*)silu_mul_quant_kernel<4, true>;
+    else
+        fn = cpt == 1 ? (const void*)silu_mul_quant_kernel<1, false>
+                      : cpt == 2 ? (const void*)silu_mul_quant_kernel<2, false> : (const void*)silu_mul_quant_kernel<4, false>;
     return status_of(launch(fn, dim3(M), dim3(threads), args, s));
 }
 

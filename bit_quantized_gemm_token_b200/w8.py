@@ -97,6 +97,8 @@ def lib():
     L.w8_quant_weight_block.argtypes = [P, I, I, P, P, I, P]
     L.w8_rmsnorm_quant.argtypes = [P, P, F, I, I, I, P, P, P]
     L.w8_silu_mul_quant.argtypes = [P, I, I, I, P, P, P]
+    L.w8_rmsnorm_quant_group.argtypes = [P, P, F, I, I, I, I, I, P, P, P]
+    L.w8_silu_mul_quant_group.argtypes = [P, I, I, I, I, I, P, P, P]
     L.w8_gemm.argtypes = [I, P, P, P, P, P, I, I, I, I, P, S, P]
     L.w8_gemm_workspace_size.argtypes = [I, I, I, I, I]
     L.w8_gemm_workspace_size.restype = S
@@ -109,7 +111,8 @@ def lib():
     L.w8_status_string.argtypes = [I]
     L.w8_status_string.restype = ctypes.c_char_p
     L.w8_version.argtypes = []
-    for fn in ("w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant", "w8_gemm",
+    for fn in ("w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant",
+               "w8_rmsnorm_quant_group", "w8_silu_mul_quant_group", "w8_gemm",
                "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
         getattr(L, fn).restype = I
     _lib = L
@@ -204,6 +207,36 @@ def w8_silu_mul_quant(gate_up, q=None, scale=None, stream=None):
         scale = torch.empty((M,), dtype=torch.float32, device=gate_up.device)
     rc = lib().w8_silu_mul_quant(_ptr(gate_up), M, I, gate_up.stride(0), _ptr(q), _ptr(scale), _stream(stream))
     _check("w8_silu_mul_quant", rc)
+    return q, scale
+
+
+def w8_rmsnorm_quant_group(x, gamma, eps=1e-6, group=128, ue8m0=False, q=None, scale=None, stream=None):
+    """rms_norm + 1x128-group fp8 quant: (e4m3 codes [M, H], scales [M, H/group])."""
+    _need(x, torch.bfloat16, "x")
+    _need(gamma, torch.bfloat16, "gamma")
+    M, H = x.shape
+    if q is None:
+        q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty((M, H // group), dtype=torch.float32, device=x.device)
+    rc = lib().w8_rmsnorm_quant_group(_ptr(x), _ptr(gamma), float(eps), M, H, x.stride(0), group, int(bool(ue8m0)),
+                                      _ptr(q), _ptr(scale), _stream(stream))
+    _check("w8_rmsnorm_quant_group", rc)
+    return q, scale
+
+
+def w8_silu_mul_quant_group(gate_up, group=128, ue8m0=False, q=None, scale=None, stream=None):
+    """silu_and_mul + 1x128-group fp8 quant: (e4m3 codes [M, I], scales [M, I/group])."""
+    _need(gate_up, torch.bfloat16, "gate_up")
+    M, I2 = gate_up.shape
+    I = I2 // 2
+    if q is None:
+        q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=gate_up.device)
+    if scale is None:
+        scale = torch.empty((M, I // group), dtype=torch.float32, device=gate_up.device)
+    rc = lib().w8_silu_mul_quant_group(_ptr(gate_up), M, I, gate_up.stride(0), group, int(bool(ue8m0)), _ptr(q),
+                                       _ptr(scale), _stream(stream))
+    _check("w8_silu_mul_quant_group", rc)
     return q, scale
 
 

@@ -171,6 +171,17 @@ W8_API int w8_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, 
  *   q e4m3 [M, I]; scale fp32 [M].  I % 8 == 0, ld % 8 == 0, 16-byte aligned. */
 W8_API int w8_silu_mul_quant(const void* gate_up, int M, int I, int ld, void* q, float* scale, w8_stream_t stream);
 
+/* Per-block fused producers for Block-FP8 ([FP8] "Kernels Helion implementados":
+ * rms_norm_per_block_quant, silu_and_mul_per_block_quant): the same fp32 rms_norm /
+ * silu_and_mul as above, then fp8 quantization with one scale per 1 x `group` block of
+ * each row (group must be 128; H or I a multiple of it), fp32 or UE8M0 (`ue8m0`) scales.
+ *   q e4m3 [M, H] or [M, I]; scale fp32 [M, H/128] or [M, I/128] (row-major).
+ * Same alignment rules and errors as the per-token producers. */
+W8_API int w8_rmsnorm_quant_group(const void* x, const void* gamma, float eps, int M, int H, int ldx, int group,
+                                  int ue8m0, void* q, float* scale, w8_stream_t stream);
+W8_API int w8_silu_mul_quant_group(const void* gate_up, int M, int I, int ld, int group, int ue8m0, void* q,
+                                   float* scale, w8_stream_t stream);
+
 /* Scaled 8-bit GEMM, out = A . W^T with the format's scales, as ONE kernel family whose
  * Standard, Split-K and Swap-AB forms are chosen by `variant` ([LIN] "Unified GEMM
  * Architecture"; [IT] paragraphs 2-3; [FP8] "Kernels Helion implementados":

@@ -52,6 +52,10 @@ def lib():
         L.orc_silu_mul_f32.restype = None
         L.orc_silu_mul_quant.argtypes = [P, i, i, i, P, P]
         L.orc_silu_mul_quant.restype = i
+        L.orc_rmsnorm_quant_group.argtypes = [P, P, f, i, i, i, i, i, P, P]
+        L.orc_rmsnorm_quant_group.restype = i
+        L.orc_silu_mul_quant_group.argtypes = [P, i, i, i, i, i, P, P]
+        L.orc_silu_mul_quant_group.restype = i
         L.orc_gemm.argtypes = [i, P, P, P, P, i, i, i, i, i, P, P, P]
         L.orc_gemm.restype = None
         L.orc_gemm_points.argtypes = [i, P, P, P, P, i, i, i, i, P, P, P]
@@ -174,6 +178,30 @@ def silu_mul_quant(xgu_bits):
     q = np.zeros((M, I), dtype=np.uint8)
     s = np.zeros((M,), dtype=np.float32)
     lib().orc_silu_mul_quant(_p(x), M, I, I2, _p(q), _p(s))
+    return q, s
+
+
+def rmsnorm_quant_group(x_bits, gamma_bits, eps, group=128, ue8m0=False):
+    x = _c(x_bits, np.uint16)
+    g = _c(gamma_bits, np.uint16)
+    M, H = x.shape
+    q = np.zeros((M, H), dtype=np.uint8)
+    s = np.zeros((M, H // group), dtype=np.float32)
+    rc = lib().orc_rmsnorm_quant_group(_p(x), _p(g), float(eps), M, H, H, group, int(bool(ue8m0)), _p(q), _p(s))
+    if rc != 0:
+        raise ValueError("orc_rmsnorm_quant_group failed: %d" % rc)
+    return q, s
+
+
+def silu_mul_quant_group(xgu_bits, group=128, ue8m0=False):
+    x = _c(xgu_bits, np.uint16)
+    M, I2 = x.shape
+    I = I2 // 2
+    q = np.zeros((M, I), dtype=np.uint8)
+    s = np.zeros((M, I // group), dtype=np.float32)
+    rc = lib().orc_silu_mul_quant_group(_p(x), M, I, I2, group, int(bool(ue8m0)), _p(q), _p(s))
+    if rc != 0:
+        raise ValueError("orc_silu_mul_quant_group failed: %d" % rc)
     return q, s
 
 

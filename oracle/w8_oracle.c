@@ -251,6 +251,39 @@ int orc_rmsnorm_quant(const uint16_t* x, const uint16_t* gamma, float eps,
     return 0;
 }
 
+/* fp8 quantization of fp32 rows v[M, K] (row-major): one scale per row (group == 0) or
+ * per 1x`group` block of a row (scale[m * (K/group) + g]), fp32 or UE8M0 scales. */
+static int orc_quant_f32_rows(const float* v, int M, int K, int group, int ue8m0, uint8_t* q, float* scale)
+{
+    if (group < 0 || (group > 0 && K % group != 0)) return -1;
+    int gsz = group ? group : K;
+    int ng = K / gsz;
+    for (int m = 0; m < M; ++m) {
+        for (int g = 0; g < ng; ++g) {
+            const float* row = v + (size_t)m * K + (size_t)g * gsz;
+            float amax = 0.0f;
+            for (int k = 0; k < gsz; ++k) amax = fmaxf(amax, fabsf(row[k]));
+            float s = orc_scale(amax, 448.0f, ue8m0);
+            scale[(size_t)m * ng + g] = s;
+            orc_encode_row(ORC_Q_FP8, row, gsz, s, q + (size_t)m * K + (size_t)g * gsz);
+        }
+    }
+    return 0;
+}
+
+/* rms_norm followed by 1x`group` fp8 quantization of the fp32 result ([FP8] "Kernels
+ * Helion implementados": rms_norm_per_block_quant; the Block-FP8 activation side). */
+int orc_rmsnorm_quant_group(const uint16_t* x, const uint16_t* gamma, float eps, int M, int H, int ldx,
+                            int group, int ue8m0, uint8_t* q, float* scale)
+{
+    float* y = (float*)malloc(sizeof(float) * (size_t)M * H);
+    if (!y) return -2;
+    orc_rmsnorm_f32(x, gamma, eps, M, H, ldx, y);
+    int rc = orc_quant_f32_rows(y, M, H, group, ue8m0, q, scale);
+    free(y);
+    return rc;
+}
+
 /* exp(x) in fp32, written for this project so that the CPU and GPU sides can agree to
  * the bit (neither may call a vendor exp).  Method: Cody & Waite argument reduction
  * (W. J. Cody, W. Waite, "Software Manual for the Elementary Functions", 1980):
@@ -301,6 +334,19 @@ void orc_silu_mul_f32(const uint16_t* xgu, int M, int I, int ld, float* h)
             h[(size_t)m * I + k] = sg * u;
         }
     }
+}
+
+/* silu_and_mul followed by 1x`group` fp8 quantization of the fp32 result ([FP8]
+ * "Kernels Helion implementados": silu_and_mul_per_block_quant). */
+int orc_silu_mul_quant_group(const uint16_t* xgu, int M, int I, int ld, int group, int ue8m0, uint8_t* q,
+                             float* scale)
+{
+    float* h = (float*)malloc(sizeof(float) * (size_t)M * I);
+    if (!h) return -2;
+    orc_silu_mul_f32(xgu, M, I, ld, h);
+    int rc = orc_quant_f32_rows(h, M, I, group, ue8m0, q, scale);
+    free(h);
+    return rc;
 }
 
 /* silu_and_mul followed by dynamic per-token fp8 quant of the fp32 result. */

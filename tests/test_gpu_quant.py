@@ -93,3 +93,24 @@ def test_quant_prefill_rows(orc):
     oq, os_ = orc.quant_rows(0, bits(x))
     assert np.array_equal(s.cpu().numpy(), os_)
     assert np.array_equal(u8(q), oq)
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("M,H", [(1, 4096), (5, 4096), (32, 5120), (300, 1024), (2, 25600), (3, 128)])
+def test_rmsnorm_quant_group_bit_exact(orc, M, H, ue8m0):
+    x = synth.activations(M, H, seed=4100 + M + H)
+    g = synth.gamma(H, seed=4101 + H)
+    q, s = w8.w8_rmsnorm_quant_group(x.cuda(), g.cuda(), 1e-6, 128, ue8m0)
+    oq, os_ = orc.rmsnorm_quant_group(bits(x), bits(g), 1e-6, 128, ue8m0)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("M,I", [(1, 12288), (3, 12288), (32, 12288), (64, 1024), (4, 25600), (2, 128)])
+def test_silu_mul_quant_group_bit_exact(orc, M, I, ue8m0):
+    xgu = synth.activations(M, 2 * I, seed=5100 + M + I)
+    q, s = w8.w8_silu_mul_quant_group(xgu.cuda(), 128, ue8m0)
+    oq, os_ = orc.silu_mul_quant_group(bits(xgu), 128, ue8m0)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)

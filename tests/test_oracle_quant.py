@@ -209,3 +209,24 @@ def test_silu_mul_quant_codes(orc):
     h = orc.silu_mul_f32(synth.bf16_bits(xgu))
     tq, ts = torch_quant(h, 0)
     assert np.array_equal(s, ts[:, 0]) and np.array_equal(q, tq)
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_rmsnorm_quant_group_codes(orc, ue8m0):
+    M, H = 4, 4096
+    x = synth.activations(M, H, seed=45)
+    g = synth.gamma(H, seed=46)
+    q, s = orc.rmsnorm_quant_group(synth.bf16_bits(x), synth.bf16_bits(g), 1e-6, 128, ue8m0)
+    y = orc.rmsnorm_f32(synth.bf16_bits(x), synth.bf16_bits(g), 1e-6)
+    tq, ts = torch_quant(y, 0, group=128, ue8m0=ue8m0)
+    assert np.array_equal(s, ts) and np.array_equal(q, tq)
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+def test_silu_mul_quant_group_codes(orc, ue8m0):
+    M, I = 3, 12288
+    xgu = synth.activations(M, 2 * I, seed=55)
+    q, s = orc.silu_mul_quant_group(synth.bf16_bits(xgu), 128, ue8m0)
+    h = orc.silu_mul_f32(synth.bf16_bits(xgu))
+    tq, ts = torch_quant(h, 0, group=128, ue8m0=ue8m0)
+    assert np.array_equal(s, ts) and np.array_equal(q, tq)
