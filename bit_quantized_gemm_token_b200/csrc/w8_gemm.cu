@@ -86,11 +86,14 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
     q.pdl = (variant & W8_V_PDL) ? 1 : 0;
     q.cluster = (variant & W8_V_CLUSTER) ? 1 : 0;
     q.bm = (variant & W8_V_BM64) ? 64 : 128;
+    q.pfix = (variant & W8_V_PFIX) ? 1 : 0;
     if (lg > 8) return W8_ERR_UNSUPPORTED;
     // the 64-row tile holds tokens: Standard form, FP8 / INT8, weight tiles of 128 or 256 rows
     if (q.bm == 64 && (q.swap || block || (tid != kTileBN128 && tid != kTileBN256))) return W8_ERR_UNSUPPORTED;
     // cluster split: 2, 4 or 8 K chunks, one cluster (portable size) per tile
     if (q.cluster && (q.stream || lg < 1 || lg > 3)) return W8_ERR_UNSUPPORTED;
+    // the parallel fixup is written for the 64-row token tile's [row][column] partials
+    if (q.pfix && (q.bm != 64 || q.cluster)) return W8_ERR_UNSUPPORTED;
     if (tid >= kNumTiles) return W8_ERR_UNSUPPORTED;
     q.bn = tile_bn(tid);
     if (block && q.bn > 64) return W8_ERR_UNSUPPORTED;   // block promotion keeps the tile in registers
@@ -143,6 +146,8 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
         q.G = (int)g;
         q.align_tiles = 1;
     }
+    // contributors of a tile wait for one another only if all CTAs can be resident at once
+    if (q.pfix && q.G > sms) return W8_ERR_UNSUPPORTED;
     // partial slots exist whenever some tile's K range can be split across CTAs (the
     // cluster split reduces through distributed shared memory instead)
     const bool partials = !q.align_tiles && !(q.G == q.tiles) && !q.cluster;   // G == tiles: one whole tile per CTA
@@ -183,6 +188,7 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     args.G = p.G;
     args.align_tiles = p.align_tiles;
     args.csplit = p.cluster ? p.split : 0;
+    args.pfix = p.pfix;
     args.w_ptr = static_cast<const uint8_t*>(W_q);
     args.stages = p.stages;
     args.pdl = p.pdl;

@@ -73,6 +73,7 @@ struct GemmArgs {
     int ld_sblk;   // K/128: row length of the block-scale matrices
     int vec_ok;    // Standard epilogue may use 16-byte stores (N % 8 == 0, out 16-byte aligned)
     int csplit;    // cluster split: the K chunks of a tile are the CTAs of one cluster (0 = off)
+    int pfix;      // 64-row token tile: split tiles are finished by all their contributors
     const uint8_t* w_ptr;   // weight codes [N, K] (for the L2 prefetch under PDL)
     const float* sA;
     const float* sW;
@@ -134,6 +135,31 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     for (uint32_t it = 1;; ++it) {
         if (probe()) return true;
         if ((it & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer_ns() - t0 > kWaitNs) {
+                *abort_flag = 1;
+                record_error(W8_ERR_DEVICE_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Poll a global counter until it reaches `target` (acquire, GPU scope), bounded like
+// wait_bounded.  Used by the parallel fixup, whose contributors are all resident.
+__device__ __forceinline__ bool wait_count(const int* p, int target, volatile int* abort_flag)
+{
+    auto probe = [&] {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        return v >= target;
+    };
+    if (probe()) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (probe()) return true;
+        if ((it & 63u) == 0) {
             if (*abort_flag) return false;
             if (ptx::globaltimer_ns() - t0 > kWaitNs) {
                 *abort_flag = 1;
@@ -225,9 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kRBytes = BM * 128;
     constexpr int kCBytes = BN * 128;
     constexpr int kStageBytes = KPS * (kRBytes + kCBytes);
-    // accumulators in TMEM: double-buffered, except for the 64-row token tile, whose single
-    // 256-column buffer leaves room for a CTA of the next kernel on the same SM
-    constexpr int kAccBufs = (BM == 64) ? 1 : 2;
+    // accumulators in TMEM, double-buffered (2 x BN <= 512 columns)
+    constexpr int kAccBufs = 2;
     constexpr uint32_t kTmemCols = (kAccBufs * BN <= 32) ? 32 : (kAccBufs * BN <= 64) ? 64 : (kAccBufs * BN <= 128) ? 128 : (kAccBufs * BN <= 256) ? 256 : 512;
     constexpr uint32_t kIdesc = instr_desc<KIND, BM, BN>();
 
@@ -281,7 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // CTA of the previous kernel holds
     uint32_t tmem = 0;
     if (warp != 0) {
-        if (warp == 1) ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+        if (warp == 1) {
+            ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+            // Dependent kernels are released only once this CTA holds its TMEM columns: a
+            // CTA of a dependent on the same SM then never takes columns this one still
+            // needs (it would hold them while waiting for this grid to finish).
+            if (lane == 0) ptx::grid_dep_launch();
+        }
         ptx::tc_fence_before();
         ptx::bar_sync(kTmemBarrier, kThreads - 32);
         ptx::tc_fence_after();
@@ -313,12 +344,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (load_c) ptx::tma_load_2d(ptx::smem_u32(c_slot(s, j)), &tmC, fb, (kb0 + j) * 128, ct * BN, pol_C);
                 }
             };
-            // With programmatic dependent launch this kernel releases its dependents at
-            // once and, before waiting for the kernels ahead of it, requests the weight
-            // boxes of the first `pre` stages (weights are never the output of work in
-            // flight; the epilogue warps prefetch the next units' weights into L2); the
-            // activation boxes follow after the wait.
-            ptx::grid_dep_launch();
+            // With programmatic dependent launch, before waiting for the kernels ahead of
+            // this one, the producer requests the weight boxes of the first `pre` stages
+            // (weights are never the output of work in flight; the epilogue warps prefetch
+            // the next units' weights into L2); the activation boxes follow after the wait.
             const int pre = a.pdl ? (int)(n < S ? n : S) : 0;
             for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap != 0, a.swap == 0, true);
             ptx::grid_dep_wait();
@@ -441,6 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16);
         const bool first_epi = (threadIdx.x == 64);
         constexpr int kAccRegs = BLOCK ? BN : 1;
+        // parallel fixup (64-row token tile): split tiles this CTA contributed to, finished
+        // after its last segment (at most its first and its last segment are split)
+        int fix_t[2] = {0, 0};
+        int nfix = 0;
         int buf = 0;
         uint32_t bphase = 0;
         bool ok = true;
@@ -664,7 +697,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(tempty + buf));
                 if (++buf == kAccBufs) { buf = 0; bphase ^= 1u; }
             }
-            if (!full_tile && a.csplit <= 1) {
+            if (!full_tile && a.csplit <= 1 && kCompact && a.pfix) {
+                // ---- parallel fixup: count this contribution, finish the tile later
+                __threadfence();
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (first_epi) atomicAdd(a.counters + t, 1);
+                if (nfix < 2) fix_t[nfix] = t;
+                ++nfix;
+            } else if (!full_tile && a.csplit <= 1) {
                 // ---- ticket: the last contributor of tile t finishes it
                 __threadfence();
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
@@ -748,6 +788,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             u += sb_hi - sb_lo;
+        }
+        if (BM == 64 && a.pfix && ok) {
+            // ---- parallel fixup.  Every contributor of a split tile has published its
+            // [row][column] partial before it waits here, so the waits end once the last
+            // one has published.  Contributor j of nc adds, for its slice of 4-column
+            // groups, the nc partials in CTA order; a second round of increments tells
+            // the last one out to reset the counter for the next call.
+            const int te = threadIdx.x - 64;
+            for (int f = 0; f < nfix && f < 2; ++f) {
+                const int t = fix_t[f];
+                const int rt = t / a.c_tiles, ct = t % a.c_tiles;
+                const int g_lo = cta_of_unit(a, (long long)t * nsb);
+                const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1);
+                const int nc = g_hi - g_lo + 1;
+                const int j = (int)blockIdx.x - g_lo;
+                bool w = true;
+                if (first_epi) w = wait_count(a.counters + t, nc, abort_flag);
+                if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) { ok = false; break; }
+                const int ncv = (a.rows_C - ct * BN < BN) ? a.rows_C - ct * BN : BN;
+                const int nrows = (a.rows_R - rt * BM < BM) ? a.rows_R - rt * BM : BM;
+                const int ng = (ncv + 3) / 4;
+                const int gl = j * ng / nc, gw = (j + 1) * ng / nc - gl;
+                for (int it = te; it < nrows * gw; it += kEpiThreads) {
+                    const int r = it / gw, cg = gl + it % gw;
+                    uint32_t v[4] = {0u, 0u, 0u, 0u};
+                    for (int cb = 0; cb < nc; cb += 8) {
+                        uint4 x[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int c = g_lo + cb + k;
+                            if (cb + k < nc) {
+                                const int sl = (unit_begin(a, c) / nsb == t) ? 0 : 1;
+                                const uint32_t* p = a.partials + ((size_t)c * 2 + sl) * (size_t)(BN * BM) +
+                                                    (size_t)r * BN + 4 * cg;
+                                x[k] = __ldcg(reinterpret_cast<const uint4*>(p));
+                            }
+                        }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (cb + k < nc) {
+                                const bool first = (cb + k == 0);
+                                v[0] = first ? x[k].x : add_words<KIND>(v[0], x[k].x);
+                                v[1] = first ? x[k].y : add_words<KIND>(v[1], x[k].y);
+                                v[2] = first ? x[k].z : add_words<KIND>(v[2], x[k].z);
+                                v[3] = first ? x[k].w : add_words<KIND>(v[3], x[k].w);
+                            }
+                        }
+                    }
+                    const int m = rt * BM + r;
+                    const float sr = (a.out_i32 == nullptr) ? __ldg(a.sA + m) : 1.0f;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        if (4 * cg + q4 < ncv) store_out<KIND, BLOCK>(a, m, ct * BN + 4 * cg + q4, v[q4], sr);
+                }
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (first_epi && atomicAdd(a.counters + t, 1) == 2 * nc - 1) a.counters[t] = 0;
+            }
         }
     }
 

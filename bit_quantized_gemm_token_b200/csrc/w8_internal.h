@@ -42,6 +42,7 @@ struct GemmPlan {
     int kps;          // 128-column K blocks per pipeline stage (1 or 2)
     int cluster;      // split_k chunks run as one thread-block cluster per tile
     int bm;           // rows of the MMA's M operand (128, or 64 for the narrow token tile)
+    int pfix;         // split tiles finished by all their contributors, a column slice each
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile

@@ -56,6 +56,17 @@ def candidates(fmt, M, N, K, quick=False):
                         else:
                             v = w8.variant(False, arg, bn, stages=stages, kps=kps, cluster=(kind == "cluster"), bm64=True)
                         out.append(v)
+        # the same with the parallel fixup of split tiles
+        for bn in (128, 256):
+            for kind, arg in [("stream", 1), ("split", 2), ("split", 4), ("split", 8)]:
+                for kps in (1, 2):
+                    for stages in ((0,) if quick else (0, 3, 4, 5)):
+                        if kind == "stream":
+                            v = w8.variant(False, 1, bn, stream=True, stages=stages, kps=kps, cps=1, bm64=True,
+                                           pfix=True)
+                        else:
+                            v = w8.variant(False, arg, bn, stages=stages, kps=kps, bm64=True, pfix=True)
+                        out.append(v)
     legal = []
     for v in out:
         try:

@@ -100,6 +100,14 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 weights in its N slot (tile 128 or 256; FP8 / INT8).  Each MMA then
  *                 consumes BN weight rows; for decode sizes this carries twice the weight
  *                 bytes per tensor-core instruction of the 128-row Swap-AB tile.
+ *   W8_V_PFIX     with W8_V_BM64 and without W8_V_CLUSTER: a tile whose K range is
+ *                 shared by several CTAs is finished by all of them together.  Each one
+ *                 publishes its partial, waits (bounded) until every contributor of the
+ *                 tile has, then adds the contributors' partials in CTA order for its own
+ *                 slice of the tile's columns.  This needs every CTA of the launch resident
+ *                 at once (as a cooperative launch does), so the launch may not exceed the
+ *                 SM count (ctas/SM must be 1).  Without it the contributor that arrives
+ *                 last adds the whole tile alone.
  *   kps           bits 20..21, 128-column K blocks carried by one pipeline stage (0 =
  *                 default: 2 for BN <= 64, else 1).  The partition unit is one stage
  *                 block, so split_k must not exceed ceil(K / (128 * kps)).
@@ -122,6 +130,7 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 #define W8_V_PDL (1 << 16)
 #define W8_V_CLUSTER (1 << 17)
 #define W8_V_BM64 (1 << 18)
+#define W8_V_PFIX (1 << 19)
 #define W8_V_KPS_SHIFT 20
 #define W8_V_CPS_SHIFT 22
 #define W8_VARIANT(swap, log2_split, tile, stream)                                            \

@@ -82,6 +82,16 @@ def test_variant_resolution_and_workspace(L):
     assert L.w8_gemm_resolve_variant(2, 8, 256, 256, w8.variant(True, bn=128)) == w8.W8_ERR_UNSUPPORTED  # block needs BN <= 64
     assert L.w8_gemm_resolve_variant(0, 8, 256, 200, 0) == w8.W8_ERR_ALIGNMENT          # K % 16
     assert L.w8_gemm_resolve_variant(2, 8, 256, 144, 0) == w8.W8_ERR_ALIGNMENT          # block K % 128
+    # parallel fixup: 64-row token tile only, no cluster, at most one CTA per SM
+    assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True)) > 0
+    assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(True, 1, 16, stream=True, pfix=True)) == \
+        w8.W8_ERR_UNSUPPORTED
+    assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(False, 2, 256, cluster=True, bm64=True, pfix=True)) == \
+        w8.W8_ERR_UNSUPPORTED
+    assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(False, 1, 256, stream=True, bm64=True, cps=2,
+                                                                   pfix=True)) == w8.W8_ERR_UNSUPPORTED
+    assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(False, 8, 128, bm64=True, pfix=True)) == \
+        w8.W8_ERR_UNSUPPORTED                                                         # 32 tiles x 8 > 148 CTAs
     # workspace: none for whole-tile partitions, some for split / balanced
     assert w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=1, bn=16)) == 0
     n = w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=4, bn=16))

@@ -35,6 +35,10 @@ VARIANTS = {
     "bm64_256_split4_pdl": w8.variant(False, 4, 256, bm64=True, stages=2, pdl=True),
     "bm64_256_cluster4": w8.variant(False, 4, 256, cluster=True, bm64=True, stages=3),
     "bm64_128_stream2": w8.variant(False, 1, 128, stream=True, bm64=True, cps=2, stages=2),
+    "bm64_256_stream_pfix": w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True),
+    "bm64_256_stream_pfix_pdl": w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True, pdl=True, kps=1, stages=5),
+    "bm64_128_split4_pfix_kps2": w8.variant(False, 4, 128, bm64=True, pfix=True, kps=2, stages=3),
+    "bm64_256_split2_pfix": w8.variant(False, 2, 256, bm64=True, pfix=True, kps=1),
 }
 
 BLOCK_OK = {"auto", "swap16", "swap32_split2", "swap16_stream", "swap64_split4", "std64_split4", "std32_split8",
@@ -129,12 +133,13 @@ def test_repeated_calls_reuse_workspace(orc):
     ws = w8.Workspace()
     A, SA, W, SW = dev_codes(Aq, 0), dev_f32(sA), dev_codes(Wq, 0), dev_f32(sW)
     outs = []
-    for v in [w8.variant(True, 8, 16), w8.variant(True, 1, 16, stream=True)] * 3:
+    for v in [w8.variant(True, 8, 16), w8.variant(True, 1, 16, stream=True),
+              w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True)] * 3:
         outs.append(w8.w8_gemm(0, A, SA, W, SW, variant=v, workspace=ws).clone())
     torch.cuda.synchronize()
     for o in outs:
         assert_bf16_close(o, ref, "repeat")
-    assert torch.equal(outs[0], outs[2]) and torch.equal(outs[1], outs[3])
+    assert torch.equal(outs[0], outs[3]) and torch.equal(outs[1], outs[4]) and torch.equal(outs[2], outs[5])
     assert int(ws.buf[:256].sum()) == 0      # counter area back to zero
     assert w8.w8_device_status(clear=True) == 0
 
