@@ -230,6 +230,19 @@ size_t w8_gemm_workspace_size(int fmt, int M, int N, int K, int variant)
     return plan.ws_bytes;
 }
 
+int w8_gemm_occupancy(int fmt, int M, int N, int K, int variant)
+{
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != W8_OK) return rc;
+    GemmPlan plan;
+    rc = resolve(fmt, M, N, K, variant, sms, &plan);
+    if (rc < 0) return rc;
+    int n = 0;
+    rc = gemm_occupancy(plan, &n);
+    return rc == W8_OK ? n : rc;
+}
+
 int w8_load_table(const char* path)
 {
     if (!path) return W8_ERR_INVALID_ARG;

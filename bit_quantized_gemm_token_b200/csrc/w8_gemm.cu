@@ -213,6 +213,22 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
 }
 
+// CTAs of the plan's kernel that fit on one SM together (registers, shared memory,
+// threads): 2 means a CTA of this GEMM can sit beside one of the same size.
+int gemm_occupancy(const GemmPlan& p, int* n)
+{
+    GemmMaps maps = {};
+    maps.occupancy = n;
+    GemmArgs args = {};
+    cudaError_t e = cudaErrorInvalidValue;
+    if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, nullptr);
+    else if (p.bm == 64)           e = launch_bm64(p, maps, args, nullptr);
+    else if (p.fmt == W8_FMT_INT8) e = launch_i8(p, maps, args, nullptr);
+    else                           e = launch_f8(p, maps, args, nullptr);
+    if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
+}
+
 // First nonzero device status word over the kernel families (each unit has its own).
 int gemm_device_status(int clear)
 {

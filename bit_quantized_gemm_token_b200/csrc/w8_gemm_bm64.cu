@@ -9,8 +9,8 @@ namespace {
 template <int BN, int KIND>
 cudaError_t launch_kps(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s)
 {
-    return p.kps == 2 ? launch_one<64, BN, KIND, false, 2>(p, m.R, m.C, a, s)
-                      : launch_one<64, BN, KIND, false, 1>(p, m.R, m.C, a, s);
+    return p.kps == 2 ? launch_one<64, BN, KIND, false, 2>(p, m, a, s)
+                      : launch_one<64, BN, KIND, false, 1>(p, m, a, s);
 }
 
 }  // namespace

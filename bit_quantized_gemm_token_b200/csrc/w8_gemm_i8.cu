@@ -8,8 +8,8 @@ namespace {
 template <int BN>
 cudaError_t launch_kps(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s)
 {
-    return p.kps == 2 ? launch_one<128, BN, KIND_I8, false, 2>(p, m.R, m.C, a, s)
-                      : launch_one<128, BN, KIND_I8, false, 1>(p, m.R, m.C, a, s);
+    return p.kps == 2 ? launch_one<128, BN, KIND_I8, false, 2>(p, m, a, s)
+                      : launch_one<128, BN, KIND_I8, false, 1>(p, m, a, s);
 }
 
 }  // namespace

@@ -858,9 +858,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 
+struct GemmMaps {
+    CUtensorMap R, C;
+    int* occupancy = nullptr;   // when set: report resident CTAs per SM instead of launching
+};
+
 template <int BM, int BN, int KIND, bool BLOCK, int KPS>
-cudaError_t launch_one(const GemmPlan& p, const CUtensorMap& tR, const CUtensorMap& tC, const GemmArgs& args,
-                       cudaStream_t s)
+cudaError_t launch_one(const GemmPlan& p, const GemmMaps& maps, const GemmArgs& args, cudaStream_t s)
 {
     auto kern = gemm_kernel<BM, BN, KIND, BLOCK, KPS>;
     // the large dynamic shared-memory limit is a per-device function attribute
@@ -876,6 +880,8 @@ cudaError_t launch_one(const GemmPlan& p, const CUtensorMap& tR, const CUtensorM
             configured[dev] = true;
         }
     }
+    if (maps.occupancy != nullptr)
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(maps.occupancy, kern, kThreads, p.smem_bytes);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.G);
     cfg.blockDim = dim3(kThreads);
@@ -897,7 +903,7 @@ cudaError_t launch_one(const GemmPlan& p, const CUtensorMap& tR, const CUtensorM
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, kern, tR, tC, args);
+    return cudaLaunchKernelEx(&cfg, kern, maps.R, maps.C, args);
 }
 
 
@@ -913,10 +919,6 @@ inline int status_word(int clear)
     }
     return v;
 }
-
-struct GemmMaps {
-    CUtensorMap R, C;
-};
 
 // per-family launchers (one translation unit each)
 cudaError_t launch_f8(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);

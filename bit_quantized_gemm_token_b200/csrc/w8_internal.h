@@ -57,6 +57,7 @@ struct GemmPlan {
 int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                 void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s);
+int gemm_occupancy(const GemmPlan& p, int* n);
 int gemm_device_status(int clear);
 
 // ---- per-shape variant table (w8_api.cu) ---------------------------------------------

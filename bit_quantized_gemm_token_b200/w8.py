@@ -114,6 +114,8 @@ def lib():
     L.w8_status_string.argtypes = [I]
     L.w8_status_string.restype = ctypes.c_char_p
     L.w8_version.argtypes = []
+    L.w8_gemm_occupancy.argtypes = [I, I, I, I, I]
+    L.w8_gemm_occupancy.restype = I
     for fn in ("w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant",
                "w8_rmsnorm_quant_group", "w8_silu_mul_quant_group", "w8_gemm",
                "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
@@ -249,6 +251,14 @@ def w8_gemm_workspace_size(fmt, M, N, K, variant=W8_VARIANT_AUTO):
     n = lib().w8_gemm_workspace_size(fmt, M, N, K, variant)
     if n == ctypes.c_size_t(-1).value:
         raise W8Error("w8_gemm_workspace_size", W8_ERR_INVALID_ARG)
+    return n
+
+
+def w8_gemm_occupancy(fmt, M, N, K, variant=W8_VARIANT_AUTO):
+    """CTAs of the selected GEMM kernel that fit on one SM together."""
+    n = lib().w8_gemm_occupancy(fmt, M, N, K, variant)
+    if n < 0:
+        raise W8Error("w8_gemm_occupancy", n)
     return n
 
 

@@ -249,6 +249,13 @@ W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int
 W8_API int w8_gemm_noalloc(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                            void* out, int M, int N, int K, int variant, w8_stream_t stream);
 
+/* CTAs of the kernel `variant` (AUTO resolved) selects for this shape that can be resident
+ * on one SM together, from its registers, shared memory and threads (the CUDA occupancy
+ * calculator).  2 or more means a CTA of the next GEMM on the stream can start, and
+ * prefetch its weights, beside one of this GEMM while this one finishes.  Returns the
+ * count (>= 0) or a negative W8_ERR_*; needs a device. */
+W8_API int w8_gemm_occupancy(int fmt, int M, int N, int K, int variant);
+
 /* Per-shape variant table (the output of the offline sweep).  Text, one entry per line:
  *   <fmt> <N> <K> <m_max> <variant as 0x hex>
  * '#' starts a comment.  AUTO picks the entry with the same (fmt, N, K) and the

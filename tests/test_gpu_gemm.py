@@ -197,3 +197,16 @@ def test_workspace_shared_across_shapes(orc):
         torch.cuda.synchronize()
         assert_bf16_close(out, ref, "shared workspace %s" % ((M, N, K),))
     assert int(ws.buf[:65536 * 4].sum()) == 0
+
+
+def test_occupancy_query():
+    """The occupancy query answers for every family; a 6-warp CTA above 128 registers
+    per thread holds an SM alone (the register file is split per scheduler)."""
+    for fmt, M, N, K, v in [(0, 1, 4096, 4096, w8.variant(True, 4, 16, cluster=True)),
+                            (1, 8, 4096, 4096, w8.variant(True, 1, 16, stream=True)),
+                            (2, 4, 6144, 4096, w8.variant(True, 1, 32, stream=True)),
+                            (0, 8, 4096, 4096, w8.variant(False, 1, 256, stream=True, bm64=True))]:
+        n = w8.w8_gemm_occupancy(fmt, M, N, K, v)
+        assert n >= 1
+    with pytest.raises(w8.W8Error):
+        w8.w8_gemm_occupancy(0, 8, 256, 256, w8.variant(True, split=4, bn=16))
