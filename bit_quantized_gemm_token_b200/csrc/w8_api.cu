@@ -107,6 +107,60 @@ int gemm_common(int fmt, const void* A_q, const float* A_scale, const void* W_q,
     return gemm_launch(plan, A_q, A_scale, W_q, W_scale, out, out_i32, workspace, ws_bytes, s);
 }
 
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Workspace of w8_linear: the GEMM's, then (two-kernel path) the codes and the scales.
+// The codes never start inside the counter area, even for a GEMM that uses no counters:
+// other calls sharing the workspace keep their tile counters there.
+size_t linear_codes_offset(const GemmPlan& p)
+{
+    const size_t counters = (size_t)kMaxCounterTiles * 4;
+    return round256(p.ws_bytes > counters ? p.ws_bytes : counters);
+}
+
+size_t linear_ws(const GemmPlan& p)
+{
+    const bool block = p.fmt >= W8_FMT_BLOCK_FP8;
+    return linear_codes_offset(p) + round256((size_t)p.M * p.K) + round256((size_t)p.M * (block ? p.kbs : 1) * 4);
+}
+
+int linear_common(int fmt, const void* x, int ldx, const void* W_q, const float* W_scale, void* out, int M, int N,
+                  int K, int variant, void* workspace, size_t ws_bytes, uint8_t* dbg_q, float* dbg_s, cudaStream_t s)
+{
+    if (!x || !W_q || !W_scale || !out) return W8_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || ldx < K) return W8_ERR_INVALID_ARG;
+    if (fmt < W8_FMT_FP8_DYN || fmt > W8_FMT_BLOCK_FP8_UE8M0) return W8_ERR_INVALID_ARG;
+    if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(W_q, 16) || !aligned(out, 2)) return W8_ERR_ALIGNMENT;
+    if (dbg_q && !aligned(dbg_q, 16)) return W8_ERR_ALIGNMENT;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != W8_OK) return rc;
+    const bool unfused = (variant & W8_V_EXPLICIT) && (variant & W8_V_UNFUSED);
+    GemmPlan plan;
+    const int v = resolve(fmt, M, N, K, variant & ~W8_V_UNFUSED, sms, &plan);
+    if (v < 0) return v;
+    if (!unfused) {
+        rc = linear_plan(fmt, M, N, K, v, sms, &plan);
+        if (rc == W8_OK) return linear_launch(plan, x, ldx, W_q, W_scale, out, workspace, ws_bytes, dbg_q, dbg_s, s);
+        if ((variant & W8_V_EXPLICIT) || dbg_q || dbg_s) return rc;
+    }
+    if (dbg_q || dbg_s) return W8_ERR_UNSUPPORTED;
+    // two kernels: the quantizer into the workspace, then the GEMM
+    rc = gemm_plan(fmt, M, N, K, v, sms, &plan);
+    if (rc != W8_OK) return rc;
+    if (workspace == nullptr || ws_bytes < linear_ws(plan)) return W8_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return W8_ERR_ALIGNMENT;
+    const bool block = fmt >= W8_FMT_BLOCK_FP8;
+    if (!block && K > kRowMaxK) return W8_ERR_UNSUPPORTED;
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    uint8_t* Aq = base + linear_codes_offset(plan);
+    float* sA = reinterpret_cast<float*>(Aq + round256((size_t)M * K));
+    rc = block ? launch_quant_group128(x, M, K, ldx, Aq, sA, fmt == W8_FMT_BLOCK_FP8_UE8M0, s)
+               : launch_quant_rows(fmt == W8_FMT_INT8 ? W8_Q_INT8 : W8_Q_FP8, x, M, K, ldx, Aq, sA, s);
+    if (rc != W8_OK) return rc;
+    return gemm_launch(plan, Aq, sA, W_q, W_scale, out, nullptr, workspace, ws_bytes, s);
+}
+
 bool row_args_ok(const void* x, int M, int K, int ldx, const void* q, const float* scale)
 {
     return x && q && scale && M > 0 && K > 0 && ldx >= K;
@@ -241,6 +295,30 @@ int w8_gemm_occupancy(int fmt, int M, int N, int K, int variant)
     int n = 0;
     rc = gemm_occupancy(plan, &n);
     return rc == W8_OK ? n : rc;
+}
+
+int w8_linear(int fmt, const void* x, int ldx, const void* W_q, const float* W_scale, void* out, int M, int N, int K,
+              int variant, void* workspace, size_t ws_bytes, w8_stream_t stream)
+{
+    return linear_common(fmt, x, ldx, W_q, W_scale, out, M, N, K, variant, workspace, ws_bytes, nullptr, nullptr,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int w8_linear_debug(int fmt, const void* x, int ldx, const void* W_q, const float* W_scale, void* out, int M, int N,
+                    int K, int variant, void* workspace, size_t ws_bytes, void* q_out, float* s_out, w8_stream_t stream)
+{
+    if (!q_out || !s_out) return W8_ERR_INVALID_ARG;
+    return linear_common(fmt, x, ldx, W_q, W_scale, out, M, N, K, variant, workspace, ws_bytes,
+                         static_cast<uint8_t*>(q_out), s_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t w8_linear_workspace_size(int fmt, int M, int N, int K, int variant)
+{
+    int sms = 0;
+    if (check_device(&sms) != W8_OK) sms = 148;
+    GemmPlan plan;
+    if (resolve(fmt, M, N, K, variant & ~W8_V_UNFUSED, sms, &plan) < 0) return (size_t)-1;
+    return linear_ws(plan);
 }
 
 int w8_load_table(const char* path)

@@ -1,0 +1,120 @@
+// w8_codes.cuh -- scalar pieces of the 8-bit quantizers shared by the quantizer kernels
+// and the GEMM's fused activation quantization: bf16 unpacking, the e4m3 / int8 encoders,
+// the scale rule and a correctly rounded quotient x / s.
+//
+// Scales and codes ("PyTorch integra Helion en vLLM para acelerar inferencia FP8",
+// section "Kernels Helion implementados"; "Helion DSL added to vLLM to autotune linear
+// inference backends", section "Unified GEMM Architecture"): s = amax / 448 (e4m3) or
+// amax / 127 (int8), an IEEE fp32 division; s = 1 for an all-zero row or group; UE8M0
+// scales are the smallest power of two not below amax / 448; codes = RNE(x / s),
+// saturating, with x / s rounded once to fp32.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+#include "w8.h"
+
+namespace w8 {
+
+constexpr float kE4M3Max = 448.0f;
+constexpr float kInt8Max = 127.0f;
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8])
+{
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xFFFF0000u);
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p)
+{
+    return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Two fp32 -> two e4m3 codes (round to nearest even, saturating); element `lo` in the
+// low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
+{
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+__device__ __forceinline__ uint32_t int8_code(float v)
+{
+    int r = __float2int_rn(v);   // ties to even; NaN -> 0
+    r = max(-127, min(127, r));
+    return static_cast<uint32_t>(r) & 0xFFu;
+}
+
+// 8 values / s -> 8 codes packed little-endian into a uint2.
+template <int QFMT>
+__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s)
+{
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(f[i], s);
+    uint2 r;
+    if (QFMT == W8_Q_FP8) {
+        r.x = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
+        r.y = e4m3x2(v[4], v[5]) | (e4m3x2(v[6], v[7]) << 16);
+    } else {
+        r.x = int8_code(v[0]) | (int8_code(v[1]) << 8) | (int8_code(v[2]) << 16) | (int8_code(v[3]) << 24);
+        r.y = int8_code(v[4]) | (int8_code(v[5]) << 8) | (int8_code(v[6]) << 16) | (int8_code(v[7]) << 24);
+    }
+    return r;
+}
+
+__device__ __forceinline__ float scale_from_amax(float amax, float qmax, bool ue8m0)
+{
+    if (!(amax > 0.0f)) return 1.0f;
+    float r = __fdiv_rn(amax, qmax);
+    if (!ue8m0) return r;
+    int e;
+    float f = frexpf(r, &e);          // r = f * 2^e exactly, f in [0.5, 1)
+    int p = (f == 0.5f) ? e - 1 : e;  // smallest power of two >= r
+    p = max(-127, min(127, p));
+    return ldexpf(1.0f, p);
+}
+
+// Correctly rounded x / s for the quantizers, without a division per element.  The row's
+// divisor is prepared once: y = RN(1 / s') with s' = s (or s * 2^64 when s is below 2^-100,
+// so that 1 / s' stays finite; x is scaled by the same exact power of two).  Per element
+// (Markstein's theorem, P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; J.-M. Muller et al.,
+// "Handbook of Floating-Point Arithmetic", ch. on division with an FMA):
+//   q0 = RN(x * y);  r = x - q0 * s' (exact, one fma);  q = RN(q0 + r * y)
+// is the correctly rounded quotient while q stays in the normal range; the sign of x is
+// copied onto q so that -0 stays -0.  Outside the normal range (|q| < 2^-126) q may differ
+// from RN(x / s) in its last bits, but every such value encodes to a zero code.  Checked
+// against __fdiv_rn for every bf16 x and every bf16 amax with |x| <= amax (amax / 448,
+// amax / 127, UE8M0): identical e4m3 and int8 codes.
+struct RowDivisor {
+    float s;    // s' (s, or s * 2^64)
+    float y;    // RN(1 / s')
+    float f;    // 1, or 2^64: the factor applied to x
+};
+
+__device__ __forceinline__ RowDivisor make_divisor(float s)
+{
+    RowDivisor d;
+    const bool tiny = s < 0x1p-100f;
+    d.f = tiny ? 0x1p64f : 1.0f;
+    d.s = __fmul_rn(s, d.f);
+    d.y = __frcp_rn(d.s);
+    return d;
+}
+
+__device__ __forceinline__ float quotient_rn(float x, const RowDivisor& d)
+{
+    const float xs = __fmul_rn(x, d.f);
+    const float q0 = __fmul_rn(xs, d.y);
+    const float r = __fmaf_rn(-q0, d.s, xs);
+    return copysignf(__fmaf_rn(r, d.y, q0), x);
+}
+
+}  // namespace w8

@@ -44,7 +44,7 @@ size_t stage_bytes(int bm, int bn, int kps) { return (size_t)kps * ((size_t)bm *
 
 size_t smem_for(int bm, int bn, int kps, int stages)
 {
-    return 1024 + (size_t)stages * stage_bytes(bm, bn, kps) + (size_t)(2 * stages + 2 * kNumAcc + 3) * 8 + 16;
+    return 1024 + (size_t)stages * stage_bytes(bm, bn, kps) + (size_t)(2 * stages + 2 * kNumAcc + 5) * 8 + 16;
 }
 
 int default_stages(int bn, int kps)
@@ -213,6 +213,86 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- fused quantize + GEMM
+namespace {
+long long host_unit_begin(const GemmPlan& q, long long g)
+{
+    if (q.align_tiles) return (g * q.tiles / q.G) * q.nsb;
+    return g * q.units / q.G;
+}
+}  // namespace
+
+int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p)
+{
+    GemmPlan q;
+    int rc = gemm_plan(fmt, M, N, K, variant, sm_count, &q);
+    if (rc != W8_OK) return rc;
+    // the activations are the narrow C operand of a Swap-AB tile holding every token
+    if (!q.swap || q.bm != 128 || q.pfix || q.c_tiles != 1 || q.bn > 64) return W8_ERR_UNSUPPORTED;
+    int rg = 0;
+    for (long long g = 0; g < q.G; ++g) {
+        int lo = 0, n = 0;
+        region_of(host_unit_begin(q, g), host_unit_begin(q, g + 1), q.nsb, q.kps, q.kbs, &lo, &n);
+        if (n > rg) rg = n;
+    }
+    // the stages carry weights only; fewer of them if the region needs the room
+    int st = q.stages;
+    while (st > 2 && fq_smem_bytes(q.bn, q.kps, st, rg) > 232448) --st;
+    if (fq_smem_bytes(q.bn, q.kps, st, rg) > 232448) return W8_ERR_UNSUPPORTED;
+    if (q.cluster && (size_t)(q.split - 1) * q.bn * q.bm * 4 > (size_t)st * q.kps * q.bm * 128) return W8_ERR_UNSUPPORTED;
+    q.stages = st;
+    q.rg_max_kb = rg;
+    q.smem_bytes = fq_smem_bytes(q.bn, q.kps, st, rg);
+    q.fq = 1;
+    *p = q;
+    return W8_OK;
+}
+
+int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, const float* W_scale, void* out,
+                  void* workspace, size_t ws_bytes, uint8_t* dbg_q, float* dbg_s, cudaStream_t s)
+{
+    if (!p.fq) return W8_ERR_INVALID_ARG;
+    if (p.ws_bytes > 0 && (workspace == nullptr || ws_bytes < p.ws_bytes)) return W8_ERR_WORKSPACE;
+    if (p.ws_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return W8_ERR_ALIGNMENT;
+    CUtensorMap tR;
+    if (!make_tmap(&tR, W_q, p.rows_R, p.K, p.bm)) return W8_ERR_CUDA;
+    GemmArgs args = {};
+    args.M = p.M; args.N = p.N; args.K = p.K;
+    args.swap = p.swap;
+    args.rows_R = p.rows_R; args.rows_C = p.rows_C;
+    args.r_tiles = p.r_tiles; args.c_tiles = p.c_tiles; args.tiles = p.tiles;
+    args.kbs = p.kbs;
+    args.nsb = p.nsb;
+    args.units = p.units;
+    args.G = p.G;
+    args.align_tiles = p.align_tiles;
+    args.csplit = p.cluster ? p.split : 0;
+    args.w_ptr = static_cast<const uint8_t*>(W_q);
+    args.stages = p.stages;
+    args.pdl = p.pdl;
+    args.ld_sblk = p.kbs;
+    args.vec_ok = 0;
+    args.sA = nullptr;
+    args.sW = W_scale;
+    args.out = static_cast<__nv_bfloat16*>(out);
+    args.out_i32 = nullptr;
+    args.counters = p.ws_bytes ? static_cast<int*>(workspace) : nullptr;
+    args.partials = p.ws_bytes ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + p.ws_counters) : nullptr;
+    args.x = static_cast<const __nv_bfloat16*>(x);
+    args.ldx = ldx;
+    args.fq_block = p.fmt >= W8_FMT_BLOCK_FP8;
+    args.fq_ue8m0 = p.fmt == W8_FMT_BLOCK_FP8_UE8M0;
+    args.rg_max_kb = p.rg_max_kb;
+    args.dbg_q = dbg_q;
+    args.dbg_s = dbg_s;
+    GemmMaps maps;
+    maps.R = tR;
+    maps.C = tR;   // the activation map is not used: the kernel writes those tiles itself
+    const cudaError_t e = launch_fq(p, maps, args, s);
+    if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
+}
+
 // CTAs of the plan's kernel that fit on one SM together (registers, shared memory,
 // threads): 2 means a CTA of this GEMM can sit beside one of the same size.
 int gemm_occupancy(const GemmPlan& p, int* n)
@@ -221,7 +301,8 @@ int gemm_occupancy(const GemmPlan& p, int* n)
     maps.occupancy = n;
     GemmArgs args = {};
     cudaError_t e = cudaErrorInvalidValue;
-    if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, nullptr);
+    if (p.fq)                      e = launch_fq(p, maps, args, nullptr);
+    else if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, nullptr);
     else if (p.bm == 64)           e = launch_bm64(p, maps, args, nullptr);
     else if (p.fmt == W8_FMT_INT8) e = launch_i8(p, maps, args, nullptr);
     else                           e = launch_f8(p, maps, args, nullptr);
@@ -233,7 +314,7 @@ int gemm_occupancy(const GemmPlan& p, int* n)
 int gemm_device_status(int clear)
 {
     int first = 0;
-    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64}) {
+    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq}) {
         const int v = f(clear);
         if (v == W8_ERR_CUDA) return v;
         if (v != 0 && first == 0) first = v;

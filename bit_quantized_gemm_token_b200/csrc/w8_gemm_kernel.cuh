@@ -37,6 +37,7 @@
 
 #include <mutex>
 
+#include "w8_codes.cuh"
 #include "w8_internal.h"
 #include "w8_ptx.cuh"
 
@@ -81,7 +82,44 @@ struct GemmArgs {
     int32_t* out_i32;
     uint32_t* partials;   // [G][2][BN][128] raw fp32 / int32 words
     int* counters;        // [tiles]
+    // fused activation quantization (Swap-AB, every token in one C tile): the CTA reads
+    // x bf16 [M, K] (row stride ldx) and writes the codes of the K blocks it needs into
+    // shared memory itself
+    const __nv_bfloat16* x;
+    int ldx;
+    int fq_block;         // 1: one scale per 1 x 128 group (Block-FP8); 0: per token
+    int fq_ue8m0;         // group scales as powers of two
+    int rg_max_kb;        // K blocks of the largest activation region over the CTAs
+    uint8_t* dbg_q;       // optional: codes of the K blocks of weight tile 0, [M, K]
+    float* dbg_s;         // optional: scales, [M] or [M, K/128]
 };
+
+// K blocks a CTA with units [u0, u1) multiplies: its own range when the units lie in one
+// tile, else every K block (a range that crosses a tile boundary wraps around in K).
+__host__ __device__ inline void region_of(long long u0, long long u1, int nsb, int kps, int kbs, int* lo, int* n)
+{
+    if (u1 <= u0) { *lo = 0; *n = 0; return; }
+    if (u0 / nsb == (u1 - 1) / nsb) {
+        const int a = (int)(u0 % nsb) * kps;
+        int b = (int)((u1 - 1) % nsb + 1) * kps;
+        if (b > kbs) b = kbs;
+        *lo = a;
+        *n = b - a;
+    } else {
+        *lo = 0;
+        *n = kbs;
+    }
+}
+
+// Shared-memory bytes of the fused-quantization form: the activation region, the stages
+// (weights only), the barriers, and the per-token / per-group scale arrays.
+__host__ __device__ inline size_t fq_smem_bytes(int bn, int kps, int stages, int rg_kb)
+{
+    const size_t region = (size_t)rg_kb * bn * 128;
+    const size_t ctrl = (size_t)(2 * stages + 2 * 2 + 5) * 8 + 16;
+    const size_t scal = (size_t)(4 * bn + 8 * bn + bn * rg_kb) * 4;
+    return 1024 + region + (size_t)stages * kps * 128 * 128 + ctrl + scal;
+}
 
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (tcgen05): K-major operand, 128-byte swizzle, rows of
@@ -186,7 +224,8 @@ __device__ __forceinline__ uint32_t add_words(uint32_t x, uint32_t y)
 // Store one output element (row i of the R tile, column j of the C tile).  `w` is the
 // raw accumulator word: unscaled (FP8/INT8) or already block-scaled (BLOCK).
 template <int KIND, bool BLOCK>
-__device__ __forceinline__ void store_out(const GemmArgs& a, int r_row, int c_row, uint32_t w, float s_row)
+__device__ __forceinline__ void store_out(const GemmArgs& a, const float* tokscale, int r_row, int c_row, uint32_t w,
+                                          float s_row)
 {
     const int m = a.swap ? c_row : r_row;
     const int n = a.swap ? r_row : c_row;
@@ -198,8 +237,9 @@ __device__ __forceinline__ void store_out(const GemmArgs& a, int r_row, int c_ro
     }
     float v = word_to_float<KIND>(w);
     if (!BLOCK) {
-        // s_row is the scale of the R-side index; the C-side scale is looked up here
-        const float s_col = a.swap ? __ldg(a.sA + m) : __ldg(a.sW + n);
+        // s_row is the scale of the R-side index; the C-side scale is looked up here (the
+        // token scales are global, or shared when the kernel quantized the activations)
+        const float s_col = a.swap ? tokscale[m] : __ldg(a.sW + n);
         v = a.swap ? __fmul_rn(__fmul_rn(v, s_col), s_row) : __fmul_rn(__fmul_rn(v, s_row), s_col);
     }
     a.out[o] = __float2bfloat16_rn(v);
@@ -214,8 +254,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 // Store 16 consecutive C-tile columns [c_base, c_base + 16) of R-tile row r_row.  In the
 // Standard form these are 16 consecutive outputs of one row: two 16-byte stores.
 template <int KIND, bool BLOCK>
-__device__ __forceinline__ void store_chunk16(const GemmArgs& a, int r_row, int c_base, const uint32_t (&v)[16],
-                                              float s_row)
+__device__ __forceinline__ void store_chunk16(const GemmArgs& a, const float* tokscale, int r_row, int c_base,
+                                              const uint32_t (&v)[16], float s_row)
 {
     if (!a.swap && a.vec_ok && a.out_i32 == nullptr && r_row < a.M && c_base + 15 < a.N) {
         float f[16];
@@ -235,8 +275,10 @@ __device__ __forceinline__ void store_chunk16(const GemmArgs& a, int r_row, int 
         return;
     }
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) store_out<KIND, BLOCK>(a, r_row, c_base + jj, v[jj], s_row);
+    for (int jj = 0; jj < 16; ++jj) store_out<KIND, BLOCK>(a, tokscale, r_row, c_base + jj, v[jj], s_row);
 }
+
+__device__ __forceinline__ bool first_epi_thread(unsigned t) { return t == 64; }
 
 // ---------------------------------------------------------------- the kernel
 // BM = rows of the MMA's M operand ("R": 128, or 64 for a narrow token tile), BN = rows
@@ -244,13 +286,15 @@ __device__ __forceinline__ void store_chunk16(const GemmArgs& a, int r_row, int 
 // "unit" of the partition is one stage block of KPS K blocks of one output tile.
 // Accumulator row r of a BM = 64 MMA lives in TMEM lane (r % 16) + 32 * (r / 16); of a
 // BM = 128 MMA in lane r.
-template <int BM, int BN, int KIND, bool BLOCK, int KPS>
+template <int BM, int BN, int KIND, bool BLOCK, int KPS, bool FQ = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC, const GemmArgs a)
 {
     constexpr int kRBytes = BM * 128;
     constexpr int kCBytes = BN * 128;
-    constexpr int kStageBytes = KPS * (kRBytes + kCBytes);
+    // with fused activation quantization the stages carry weights only; the activation
+    // codes sit in a region of their own, written once by the epilogue warps
+    constexpr int kStageBytes = KPS * (kRBytes + (FQ ? 0 : kCBytes));
     // accumulators in TMEM, double-buffered (2 x BN <= 512 columns)
     constexpr int kAccBufs = 2;
     constexpr uint32_t kTmemCols = (kAccBufs * BN <= 32) ? 32 : (kAccBufs * BN <= 64) ? 64 : (kAccBufs * BN <= 128) ? 128 : (kAccBufs * BN <= 256) ? 256 : 512;
@@ -259,22 +303,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = a.stages;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * kStageBytes);
+    uint8_t* region = smem;   // FQ: activation codes [K block][BN rows x 128 B], 128-byte swizzled
+    uint8_t* sbase = smem + (FQ ? (size_t)a.rg_max_kb * kCBytes : 0);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sbase + (size_t)S * kStageBytes);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
     uint64_t* tempty = tfull + kNumAcc;
     uint64_t* drain = tempty + kNumAcc;
     uint64_t* red_full = drain + 1;   // cluster split (rank 0): partials of the other ranks have landed
     uint64_t* red_go = red_full + 1;  // cluster split (ranks 1..): rank 0's stage memory is free
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_go + 1);
+    uint64_t* a_ready = red_go + 1;   // FQ: the activation region is written
+    uint64_t* amax_full = a_ready + 1;   // FQ, cluster split: the other ranks' partial row maxima landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(amax_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* ticket = reinterpret_cast<volatile int*>(tmem_slot + 2);
+    // FQ scale arrays: per token scale, divisor (s', 1/s', factor), partial maxima of every
+    // cluster rank, and the group scales of the region
+    float* s_tok = reinterpret_cast<float*>(tmem_slot + 4);
+    float* s_div = s_tok + BN;                                   // [3][BN]
+    uint32_t* amax_slots = reinterpret_cast<uint32_t*>(s_div + 3 * BN);   // [8][BN]
+    float* s_blk = reinterpret_cast<float*>(amax_slots + 8 * BN);          // [BN][rg_max_kb]
     // cluster split: [csplit - 1][BN columns][BM rows] partial words, written into rank 0's
     // stage memory once its last MMA has completed (the stages are free by then)
-    uint32_t* red_buf = reinterpret_cast<uint32_t*>(smem);
+    uint32_t* red_buf = reinterpret_cast<uint32_t*>(sbase);
     // stage s: R slots [KPS][128 x 128 B], then C slots [KPS][BN x 128 B]; all 1024-aligned
-    auto r_slot = [&](int s, int j) { return smem + (size_t)s * kStageBytes + (size_t)j * kRBytes; };
-    auto c_slot = [&](int s, int j) { return smem + (size_t)s * kStageBytes + (size_t)KPS * kRBytes + (size_t)j * kCBytes; };
+    auto r_slot = [&](int s, int j) { return sbase + (size_t)s * kStageBytes + (size_t)j * kRBytes; };
+    auto c_slot = [&](int s, int j) { return sbase + (size_t)s * kStageBytes + (size_t)KPS * kRBytes + (size_t)j * kCBytes; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -290,6 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(ptx::smem_u32(drain), 1);
         ptx::mbar_init(ptx::smem_u32(red_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * kEpiThreads : 1u);
         ptx::mbar_init(ptx::smem_u32(red_go), 1);
+        ptx::mbar_init(ptx::smem_u32(a_ready), 1);
+        ptx::mbar_init(ptx::smem_u32(amax_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * kEpiThreads : 1u);
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -338,10 +394,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nkb = (kbs - kb0 < KPS) ? kbs - kb0 : KPS;
                 const int rt = t / a.c_tiles, ct = t % a.c_tiles;
                 const uint32_t fb = ptx::smem_u32(full + s);
-                if (expect) ptx::mbar_arrive_expect_tx(fb, (uint32_t)(nkb * (kRBytes + kCBytes)));
+                if (expect) ptx::mbar_arrive_expect_tx(fb, (uint32_t)(nkb * (kRBytes + (FQ ? 0 : kCBytes))));
                 for (int j = 0; j < nkb; ++j) {
                     if (load_r) ptx::tma_load_2d(ptx::smem_u32(r_slot(s, j)), &tmR, fb, (kb0 + j) * 128, rt * BM, pol_R);
-                    if (load_c) ptx::tma_load_2d(ptx::smem_u32(c_slot(s, j)), &tmC, fb, (kb0 + j) * 128, ct * BN, pol_C);
+                    if (load_c && !FQ) ptx::tma_load_2d(ptx::smem_u32(c_slot(s, j)), &tmC, fb, (kb0 + j) * 128, ct * BN, pol_C);
                 }
             };
             // With programmatic dependent launch, before waiting for the kernels ahead of
@@ -351,7 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int pre = a.pdl ? (int)(n < S ? n : S) : 0;
             for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap != 0, a.swap == 0, true);
             ptx::grid_dep_wait();
-            for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap == 0, a.swap != 0, false);
+            if (!FQ)
+                for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap == 0, a.swap != 0, false);
             long long issued = pre;
             int stage = pre % S;
             uint32_t phase = (pre == S) ? 1u : 0u;
@@ -381,6 +438,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0, buf = 0;
         uint32_t phase = 0, bphase = 0;
         bool ok = true;
+        int rg_lo = 0, rg_n = 0;
+        if (FQ) {
+            // the activation codes come from this CTA's epilogue warps
+            region_of(u0, u1, nsb, KPS, kbs, &rg_lo, &rg_n);
+            if (lane == 0) {
+                ok = wait_bounded(ptx::smem_u32(a_ready), 0, abort_flag);
+                ptx::tc_fence_after();
+            }
+            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        }
         for (long long u = u0; u < u1 && ok; ++u) {
             const int sb = (int)(u % nsb);
             const int kb0 = sb * KPS;
@@ -406,7 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (!ok) break;
                         }
                         const uint64_t dR = smem_desc(ptx::smem_u32(r_slot(stage, j)));
-                        const uint64_t dC = smem_desc(ptx::smem_u32(c_slot(stage, j)));
+                        const uint64_t dC = FQ ? smem_desc(ptx::smem_u32(region + (size_t)(kb0 + j - rg_lo) * kCBytes))
+                                               : smem_desc(ptx::smem_u32(c_slot(stage, j)));
                         const uint32_t d_tmem = tmem + (uint32_t)(b * BN);
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -463,6 +531,137 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         ptx::grid_dep_wait();
+        // token scales: global, or (FQ) the ones this CTA computes below
+        const float* tokscale = FQ ? s_tok : a.sA;
+        int rg_lo = 0, rg_n = 0;
+        bool fq_ok = true;
+        if (FQ) {
+            // ---- fused activation quantization: row (or group) maxima, scales, then the
+            // codes of every K block this CTA multiplies, written 128-byte swizzled into the
+            // region the MMA reads in place of a TMA-loaded activation tile
+            region_of(u0, u1, nsb, KPS, kbs, &rg_lo, &rg_n);
+            const int te = threadIdx.x - 64;
+            const int M = a.M, K = a.K;
+            if (!a.fq_block) {
+                // per-token maxima: over this rank's K range when the cluster's ranks
+                // together cover the tile's K (cluster split), else over the whole row
+                const bool part = a.csplit > 1;
+                const int k_lo = part ? rg_lo * 128 : 0;
+                const int k_hi = part ? min((rg_lo + rg_n) * 128, K) : K;
+                const int nch = (k_hi - k_lo) >> 3;
+                const uint32_t rank = part ? ptx::cluster_ctarank() : 0u;
+                for (int m = te >> 5; m < M; m += kEpiThreads / 32) {
+                    const __nv_bfloat16* xr = a.x + (size_t)m * a.ldx + k_lo;
+                    float mx = 0.0f;
+#pragma unroll 4
+                    for (int c = lane; c < nch; c += 32) {
+                        float f[8];
+                        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(xr + (size_t)c * 8)), f);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(f[i]));
+                    }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                    if (lane == 0) amax_slots[rank * BN + m] = __float_as_uint(mx);
+                }
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (part) {
+                    // every rank sends its partial maxima to the others (distributed shared
+                    // memory) and arrives on their barriers; each thread arrives itself
+                    for (int m = te; m < M; m += kEpiThreads)
+                        for (int r = 0; r < a.csplit; ++r)
+                            if ((uint32_t)r != rank)
+                                ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(amax_slots + rank * BN + m), (uint32_t)r),
+                                                    amax_slots[rank * BN + m]);
+                    for (int r = 0; r < a.csplit; ++r)
+                        if ((uint32_t)r != rank) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(amax_full), (uint32_t)r));
+                    const bool w = wait_bounded<true>(ptx::smem_u32(amax_full), 0, abort_flag);
+                    if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) fq_ok = false;
+                }
+                if (fq_ok) {
+                    const int nslots = part ? a.csplit : 1;
+                    for (int m = te; m < BN; m += kEpiThreads) {
+                        float amax = 0.0f;
+                        if (m < M)
+                            for (int r = 0; r < nslots; ++r) amax = fmaxf(amax, __uint_as_float(amax_slots[r * BN + m]));
+                        const float s = scale_from_amax(amax, KIND == KIND_I8 ? kInt8Max : kE4M3Max, false);
+                        const RowDivisor d = make_divisor(s);
+                        s_tok[m] = s;
+                        s_div[m] = d.s;
+                        s_div[BN + m] = d.y;
+                        s_div[2 * BN + m] = d.f;
+                        if (a.dbg_s != nullptr && blockIdx.x == 0 && m < M) a.dbg_s[m] = s;
+                    }
+                    ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                }
+            }
+            if (fq_ok) {
+                // K blocks of weight tile 0 that this CTA multiplies (for the optional copy
+                // of the codes)
+                const int dbg_lo = (u0 < nsb) ? (int)u0 * KPS : kbs;
+                const int dbg_hi = (u0 < nsb) ? (int)min(u1, (long long)nsb) * KPS : kbs;
+                // items: (row, K block, 16-code chunk); the 8 chunks of one row's K block
+                // are 8 consecutive lanes
+                const int total = BN * rg_n * 8;
+                for (int it = te; it < total; it += kEpiThreads) {
+                    const int c16 = it & 7;
+                    const int kbl = (it >> 3) % rg_n;
+                    const int m = (it >> 3) / rg_n;
+                    const int kb = rg_lo + kbl;
+                    const int k0 = kb * 128 + c16 * 16;
+                    const bool live = m < M && k0 < K;
+                    float f[16];
+                    if (live) {
+                        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)m * a.ldx + k0);
+                        float lo[8], hi[8];
+                        unpack_bf16x8(__ldg(src), lo);
+                        unpack_bf16x8(__ldg(src + 1), hi);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) { f[i] = lo[i]; f[8 + i] = hi[i]; }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) f[i] = 0.0f;
+                    }
+                    RowDivisor d;
+                    float s = 1.0f;
+                    if (a.fq_block) {
+                        // one scale per 1 x 128 group: the maximum over the group's 8 lanes
+                        float mx = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(f[i]));
+#pragma unroll
+                        for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                        s = scale_from_amax(mx, kE4M3Max, a.fq_ue8m0 != 0);
+                        d = make_divisor(s);
+                        if (c16 == 0) s_blk[m * a.rg_max_kb + kbl] = s;
+                        if (c16 == 0 && a.dbg_s != nullptr && m < M && kb >= dbg_lo && kb < dbg_hi)
+                            a.dbg_s[(size_t)m * kbs + kb] = s;
+                    } else {
+                        d.s = s_div[m];
+                        d.y = s_div[BN + m];
+                        d.f = s_div[2 * BN + m];
+                    }
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const float q0 = quotient_rn(f[4 * g], d), q1 = quotient_rn(f[4 * g + 1], d);
+                        const float q2 = quotient_rn(f[4 * g + 2], d), q3 = quotient_rn(f[4 * g + 3], d);
+                        w4[g] = (KIND == KIND_I8)
+                                    ? (int8_code(q0) | (int8_code(q1) << 8) | (int8_code(q2) << 16) | (int8_code(q3) << 24))
+                                    : (e4m3x2(q0, q1) | (e4m3x2(q2, q3) << 16));
+                    }
+                    const uint4 codes = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    *reinterpret_cast<uint4*>(region + (size_t)kbl * kCBytes + (size_t)m * 128 + (size_t)((c16 ^ (m & 7)) << 4)) =
+                        codes;
+                    if (a.dbg_q != nullptr && live && kb >= dbg_lo && kb < dbg_hi)
+                        *reinterpret_cast<uint4*>(a.dbg_q + (size_t)m * K + k0) = codes;
+                }
+                // the tensor core reads the region through the async proxy
+                ptx::fence_proxy_async_smem();
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (first_epi_thread(threadIdx.x)) ptx::mbar_arrive(ptx::smem_u32(a_ready));
+            }
+        }
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         // row of the R tile held by this thread (BM = 64: lanes 16..31 of a quadrant hold none)
         const int i = (BM == 128) ? q * 32 + lane : q * 16 + (lane & 15);
@@ -476,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nfix = 0;
         int buf = 0;
         uint32_t bphase = 0;
-        bool ok = true;
+        bool ok = fq_ok;
         for (long long u = u0; u < u1 && ok;) {
             const int t = (int)(u / nsb);
             const int sb_lo = (int)(u % nsb);
@@ -513,7 +712,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int h = 0; h < (BN + 31) / 32; ++h) {
                             const int jc = h * 32 + lane;
                             const int col = ct * BN + jc;
-                            sa_l[h] = (jc < BN && col < a.rows_C) ? __ldg(a.sA + (size_t)col * a.ld_sblk + kb) : 0.0f;
+                            sa_l[h] = (jc < BN && col < a.rows_C)
+                                          ? (FQ ? s_blk[col * a.rg_max_kb + (kb - rg_lo)] : __ldg(a.sA + (size_t)col * a.ld_sblk + kb))
+                                          : 0.0f;
                         }
                     } else {
                         const float sa = (r_row < a.rows_R) ? __ldg(a.sA + (size_t)r_row * a.ld_sblk + kb) : 0.0f;
@@ -586,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto finish = [&](int r, int col, uint32_t w) {
                 const int m = rt * BM + r;
                 const float sr = (a.out_i32 == nullptr) ? __ldg(a.sA + m) : 1.0f;
-                store_out<KIND, BLOCK>(a, m, ct * BN + col, w, sr);
+                store_out<KIND, BLOCK>(a, tokscale, m, ct * BN + col, w, sr);
             };
             if (kCompact && a.csplit > 1) {
                 // ---- cluster split, 64-row token tile: every rank's real rows go to rank 0's
@@ -666,7 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int jj = 0; jj < 16; ++jj)
                                 v[jj] = add_words<BLOCK ? KIND_F8 : KIND>(v[jj], src[(c0 + jj) * BM + i]);
                         }
-                        store_chunk16<KIND, BLOCK>(a, r_row, ct * BN + c0, v, s_row);
+                        store_chunk16<KIND, BLOCK>(a, tokscale, r_row, ct * BN + c0, v, s_row);
                     }
                 }
             } else if (full_tile) {
@@ -676,7 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (c0 >= ncv) break;
                     uint32_t v[16];
                     fetch16(c0, v);
-                    store_chunk16<KIND, BLOCK>(a, r_row, ct * BN + c0, v, s_row);
+                    store_chunk16<KIND, BLOCK>(a, tokscale, r_row, ct * BN + c0, v, s_row);
                 }
             } else {
                 // ---- partial: publish to this CTA's slot ([column][row] words, coalesced)
@@ -782,7 +983,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                             }
                         }
-                        store_chunk16<KIND, BLOCK>(a, r_row, ct * BN + c0, v, s_row);
+                        store_chunk16<KIND, BLOCK>(a, tokscale, r_row, ct * BN + c0, v, s_row);
                     }
                     if (first_epi) a.counters[t] = 0;   // leave the counter ready for the next call
                 }
@@ -840,7 +1041,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float sr = (a.out_i32 == nullptr) ? __ldg(a.sA + m) : 1.0f;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        if (4 * cg + q4 < ncv) store_out<KIND, BLOCK>(a, m, ct * BN + 4 * cg + q4, v[q4], sr);
+                        if (4 * cg + q4 < ncv) store_out<KIND, BLOCK>(a, tokscale, m, ct * BN + 4 * cg + q4, v[q4], sr);
                 }
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
                 if (first_epi && atomicAdd(a.counters + t, 1) == 2 * nc - 1) a.counters[t] = 0;
@@ -863,10 +1064,10 @@ struct GemmMaps {
     int* occupancy = nullptr;   // when set: report resident CTAs per SM instead of launching
 };
 
-template <int BM, int BN, int KIND, bool BLOCK, int KPS>
+template <int BM, int BN, int KIND, bool BLOCK, int KPS, bool FQ = false>
 cudaError_t launch_one(const GemmPlan& p, const GemmMaps& maps, const GemmArgs& args, cudaStream_t s)
 {
-    auto kern = gemm_kernel<BM, BN, KIND, BLOCK, KPS>;
+    auto kern = gemm_kernel<BM, BN, KIND, BLOCK, KPS, FQ>;
     // the large dynamic shared-memory limit is a per-device function attribute
     static bool configured[64] = {};
     static std::mutex mu;
@@ -925,10 +1126,12 @@ cudaError_t launch_f8(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, c
 cudaError_t launch_i8(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_block(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_bm64(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_fq(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 int status_f8(int clear);
 int status_i8(int clear);
 int status_block(int clear);
 int status_bm64(int clear);
+int status_fq(int clear);
 
 }  // namespace gemm
 }  // namespace w8

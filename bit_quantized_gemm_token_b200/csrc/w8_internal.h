@@ -43,6 +43,8 @@ struct GemmPlan {
     int cluster;      // split_k chunks run as one thread-block cluster per tile
     int bm;           // rows of the MMA's M operand (128, or 64 for the narrow token tile)
     int pfix;         // split tiles finished by all their contributors, a column slice each
+    int fq;           // the kernel quantizes the activations itself (w8_linear)
+    int rg_max_kb;    // fq: K blocks of the largest activation region
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile
@@ -58,6 +60,13 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                 void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s);
 int gemm_occupancy(const GemmPlan& p, int* n);
+// plan of the fused quantize + GEMM form of `variant`: Swap-AB with every token in one
+// narrow tile; W8_ERR_UNSUPPORTED when the variant has no such form
+int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);
+// fused launch: x bf16 [M, K] (row stride ldx) is quantized inside the GEMM kernel;
+// dbg_q / dbg_s (optional) receive the codes and scales of weight tile 0's K blocks
+int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, const float* W_scale, void* out,
+                  void* workspace, size_t ws_bytes, uint8_t* dbg_q, float* dbg_s, cudaStream_t s);
 int gemm_device_status(int clear);
 
 // ---- per-shape variant table (w8_api.cu) ---------------------------------------------

@@ -21,75 +21,12 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "w8_codes.cuh"
 #include "w8_internal.h"
 #include "w8_ptx.cuh"
 
 namespace w8 {
 namespace {
-
-constexpr float kE4M3Max = 448.0f;
-constexpr float kInt8Max = 127.0f;
-
-__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8])
-{
-    f[0] = __uint_as_float(v.x << 16);
-    f[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    f[2] = __uint_as_float(v.y << 16);
-    f[3] = __uint_as_float(v.y & 0xFFFF0000u);
-    f[4] = __uint_as_float(v.z << 16);
-    f[5] = __uint_as_float(v.z & 0xFFFF0000u);
-    f[6] = __uint_as_float(v.w << 16);
-    f[7] = __uint_as_float(v.w & 0xFFFF0000u);
-}
-
-__device__ __forceinline__ uint4 ld_nc_v4(const void* p)
-{
-    return __ldg(reinterpret_cast<const uint4*>(p));
-}
-
-// Two fp32 -> two e4m3 codes (round to nearest even, saturating); element `lo` in the
-// low byte.
-__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi)
-{
-    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
-}
-
-__device__ __forceinline__ uint32_t int8_code(float v)
-{
-    int r = __float2int_rn(v);   // ties to even; NaN -> 0
-    r = max(-127, min(127, r));
-    return static_cast<uint32_t>(r) & 0xFFu;
-}
-
-// 8 values / s -> 8 codes packed little-endian into a uint2.
-template <int QFMT>
-__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s)
-{
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(f[i], s);
-    uint2 r;
-    if (QFMT == W8_Q_FP8) {
-        r.x = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
-        r.y = e4m3x2(v[4], v[5]) | (e4m3x2(v[6], v[7]) << 16);
-    } else {
-        r.x = int8_code(v[0]) | (int8_code(v[1]) << 8) | (int8_code(v[2]) << 16) | (int8_code(v[3]) << 24);
-        r.y = int8_code(v[4]) | (int8_code(v[5]) << 8) | (int8_code(v[6]) << 16) | (int8_code(v[7]) << 24);
-    }
-    return r;
-}
-
-__device__ __forceinline__ float scale_from_amax(float amax, float qmax, bool ue8m0)
-{
-    if (!(amax > 0.0f)) return 1.0f;
-    float r = __fdiv_rn(amax, qmax);
-    if (!ue8m0) return r;
-    int e;
-    float f = frexpf(r, &e);          // r = f * 2^e exactly, f in [0.5, 1)
-    int p = (f == 0.5f) ? e - 1 : e;  // smallest power of two >= r
-    p = max(-127, min(127, p));
-    return ldexpf(1.0f, p);
-}
 
 __device__ __forceinline__ float warp_max(float v)
 {

@@ -40,6 +40,7 @@ W8_V_PDL = 1 << 16
 W8_V_CLUSTER = 1 << 17
 W8_V_BM64 = 1 << 18
 W8_V_PFIX = 1 << 19
+W8_V_UNFUSED = 1 << 24
 W8_V_KPS_SHIFT = 20
 W8_V_CPS_SHIFT = 22
 TILE_BN = {16: 0, 32: 1, 64: 2, 128: 3, 256: 4}
@@ -114,9 +115,14 @@ def lib():
     L.w8_status_string.argtypes = [I]
     L.w8_status_string.restype = ctypes.c_char_p
     L.w8_version.argtypes = []
+    L.w8_linear.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P]
+    L.w8_linear_debug.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P, P, P]
+    L.w8_linear_workspace_size.argtypes = [I, I, I, I, I]
+    L.w8_linear_workspace_size.restype = S
     L.w8_gemm_occupancy.argtypes = [I, I, I, I, I]
     L.w8_gemm_occupancy.restype = I
-    for fn in ("w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant",
+    for fn in ("w8_linear", "w8_linear_debug",
+               "w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant",
                "w8_rmsnorm_quant_group", "w8_silu_mul_quant_group", "w8_gemm",
                "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
         getattr(L, fn).restype = I
@@ -315,6 +321,49 @@ def w8_gemm(fmt, A_q, A_scale, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, 
                        _stream(stream))
     _check("w8_gemm", rc)
     return out
+
+
+def w8_linear_workspace_size(fmt, M, N, K, variant=W8_VARIANT_AUTO):
+    n = lib().w8_linear_workspace_size(fmt, M, N, K, variant)
+    if n == ctypes.c_size_t(-1).value:
+        raise W8Error("w8_linear_workspace_size", W8_ERR_INVALID_ARG)
+    return n
+
+
+def w8_linear(fmt, x, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
+    """out[M, N] (bf16) = scaled quant(x) . W_q^T: x bf16 [M, K] quantized per token (or
+    per 1 x 128 group for Block-FP8) and multiplied in one call (one kernel when the
+    variant has a fused form)."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = W_q.shape[0]
+    if W_q.shape[1] != K:
+        raise ValueError("K mismatch")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _need(out, torch.bfloat16, "out")
+    nbytes = w8_linear_workspace_size(fmt, M, N, K, variant)
+    wp, wn = _workspace(workspace, x.device, nbytes)
+    rc = lib().w8_linear(fmt, _ptr(x), x.stride(0), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp, wn,
+                         _stream(stream))
+    _check("w8_linear", rc)
+    return out
+
+
+def w8_linear_debug(fmt, x, W_q, W_scale, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
+    """Fused w8_linear that also returns the codes [M, K] (uint8) and scales it computed."""
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = W_q.shape[0]
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    q = torch.zeros((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.zeros((M, K // 128) if fmt >= W8_FMT_BLOCK_FP8 else (M,), dtype=torch.float32, device=x.device)
+    nbytes = w8_linear_workspace_size(fmt, M, N, K, variant)
+    wp, wn = _workspace(workspace, x.device, nbytes)
+    rc = lib().w8_linear_debug(fmt, _ptr(x), x.stride(0), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp,
+                               wn, _ptr(q), _ptr(s), _stream(stream))
+    _check("w8_linear_debug", rc)
+    return out, q, s
 
 
 def w8_gemm_i32_debug(A_q, W_q, acc=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):

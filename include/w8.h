@@ -131,6 +131,7 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 #define W8_V_CLUSTER (1 << 17)
 #define W8_V_BM64 (1 << 18)
 #define W8_V_PFIX (1 << 19)
+#define W8_V_UNFUSED (1 << 24)
 #define W8_V_KPS_SHIFT 20
 #define W8_V_CPS_SHIFT 22
 #define W8_VARIANT(swap, log2_split, tile, stream)                                            \
@@ -231,6 +232,39 @@ W8_API int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant);
  * of the integer path. */
 W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int N, int K, int variant,
                       void* workspace, size_t ws_bytes, w8_stream_t stream);
+
+/* Quantize-and-multiply in one call: out = w8_gemm(fmt, quant(x), W) for a bf16
+ * activation x [M, K] (row stride ldx elements), with quant the per-token quantizer of
+ * w8_quant_per_token for FP8-dynamic (e4m3) and W8A8-INT8 (int8), or its 1 x 128 group
+ * form for Block-FP8 (fp32 or UE8M0 scales).  The result is bit-identical to the two
+ * calls with the same variant.  ("PyTorch integra Helion en vLLM para acelerar
+ * inferencia FP8", section "Patron de fusion del forward pass": the quantizer fused
+ * into its neighbour; here the neighbour is the GEMM itself.)
+ *   When the resolved variant is Swap-AB with every token in one narrow tile (M <= BN
+ *   <= 64), ONE kernel does both: each CTA reads x, computes the row (or group) maxima
+ *   -- over its own K range, exchanged between the ranks of a cluster split, else over
+ *   the whole row -- and writes the codes of the K blocks it multiplies straight into
+ *   shared memory, where the tensor core reads them; the quotient x / s is correctly
+ *   rounded without a division per element (same codes as the quantizer kernels).
+ *   Otherwise (larger M, Standard tiles) the quantizer kernel runs first into the
+ *   workspace, then the GEMM.  AUTO picks the table's variant and the fused form when it
+ *   exists; an explicit variant must have a fused form unless it carries W8_V_UNFUSED,
+ *   which forces the two-kernel path.
+ * x: 16-byte aligned, ldx >= K and a multiple of 8; K as for w8_gemm.  workspace /
+ * ws_bytes: at least w8_linear_workspace_size (same rules as w8_gemm's workspace; the
+ * two-kernel path keeps the codes and scales there, past the 256 KiB counter area).
+ * Errors: as w8_gemm. */
+W8_API int w8_linear(int fmt, const void* x, int ldx, const void* W_q, const float* W_scale, void* out, int M, int N,
+                     int K, int variant, void* workspace, size_t ws_bytes, w8_stream_t stream);
+W8_API size_t w8_linear_workspace_size(int fmt, int M, int N, int K, int variant);
+
+/* The fused form of w8_linear that also writes the codes it computed for the K blocks of
+ * weight tile 0 (all of K) to q_out [M, K] (16-byte aligned) and the scales to s_out
+ * ([M], or [M, K/128] for Block-FP8).  For checking the fused quantization bit for bit;
+ * W8_ERR_UNSUPPORTED when the variant has no fused form. */
+W8_API int w8_linear_debug(int fmt, const void* x, int ldx, const void* W_q, const float* W_scale, void* out, int M,
+                           int N, int K, int variant, void* workspace, size_t ws_bytes, void* q_out, float* s_out,
+                           w8_stream_t stream);
 
 /* w8_gemm for callers that cannot allocate device memory.  (An addition of this
  * library: the pages describe no counterpart.)  Some callers cannot provide the
