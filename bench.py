@@ -203,9 +203,11 @@ class Workload:
                 self.A[(M, K, N)] = (torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
                                      torch.empty((M,), dtype=torch.float32, device=dev))
                 self.OUT[(M, K, N)] = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        nb = max(w8.w8_gemm_workspace_size(w8.W8_FMT_FP8_DYN, M, N, K, w8.W8_V_PDL)
+        nb = max(max(w8.w8_gemm_workspace_size(w8.W8_FMT_FP8_DYN, M, N, K, w8.W8_V_PDL),
+                     w8.w8_linear_workspace_size(w8.W8_FMT_FP8_DYN, M, N, K, w8.W8_V_PDL))
                  for M in ms for (K, N) in shapes)
         self.ws = w8.Workspace(dev, nb)
+        self.path = "pair"
         torch.cuda.synchronize()
 
     def rotate(self, ncopy):
@@ -229,6 +231,15 @@ class Workload:
         w8 = self.w8
         v = w8.W8_VARIANT_AUTO | w8.W8_V_PDL
         n = 0
+        if self.path == "linear" and quant and gemm:
+            # quantize + GEMM per layer through w8_linear: the quantizer and the GEMM, or one
+            # kernel where the table asks for the fused form
+            for M, K, N, c in self.order():
+                Wq, sW = self.W[(K, N, c)]
+                w8.w8_linear(w8.W8_FMT_FP8_DYN, self.X[(M, K, N)], Wq, sW, out=self.OUT[(M, K, N)], variant=v,
+                             workspace=self.ws)
+                n += 1 if (w8.w8_linear_resolve(0, M, N, K, v) & w8.W8_V_FUSED) else 2
+            return n
         for M, K, N, c in self.order():
             q, s = self.A[(M, K, N)]
             if quant:
@@ -389,6 +400,7 @@ def run_ours(args):
         shapes, ms = [(K, N)], [args.m]
         workload = "single FP8-dynamic quant + GEMM, M=%d, KxN=%dx%d" % (args.m, K, N)
     wl = Workload(dev, shapes, ms, seed=1234 + 1 + rank)
+    wl.path = args.path
     gb, qb = step_bytes(shapes, ms)
 
     try:
@@ -501,6 +513,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--detail", action="store_true", help="also time every (shape, M) GEMM alone")
+    ap.add_argument("--path", default="pair", choices=["pair", "linear"],
+                    help="per layer: quantizer + GEMM calls (pair) or w8_linear (fused where it can)")
     ap.add_argument("--single", default="", help="KxN: time one shape only (profiling case)")
     ap.add_argument("--m", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")

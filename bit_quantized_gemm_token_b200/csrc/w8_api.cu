@@ -135,16 +135,17 @@ int linear_common(int fmt, const void* x, int ldx, const void* W_q, const float*
     int sms = 0;
     int rc = check_device(&sms);
     if (rc != W8_OK) return rc;
-    const bool unfused = (variant & W8_V_EXPLICIT) && (variant & W8_V_UNFUSED);
     GemmPlan plan;
-    const int v = resolve(fmt, M, N, K, variant & ~W8_V_UNFUSED, sms, &plan);
+    int v = resolve(fmt, M, N, K, variant, sms, &plan);
     if (v < 0) return v;
-    if (!unfused) {
+    // the one-kernel form when asked for (explicitly, or by the table's entry for AUTO)
+    const bool fused = (v & W8_V_FUSED) || dbg_q || dbg_s;
+    v &= ~W8_V_FUSED;
+    if (fused) {
         rc = linear_plan(fmt, M, N, K, v, sms, &plan);
-        if (rc == W8_OK) return linear_launch(plan, x, ldx, W_q, W_scale, out, workspace, ws_bytes, dbg_q, dbg_s, s);
-        if ((variant & W8_V_EXPLICIT) || dbg_q || dbg_s) return rc;
+        if (rc != W8_OK) return rc;
+        return linear_launch(plan, x, ldx, W_q, W_scale, out, workspace, ws_bytes, dbg_q, dbg_s, s);
     }
-    if (dbg_q || dbg_s) return W8_ERR_UNSUPPORTED;
     // two kernels: the quantizer into the workspace, then the GEMM
     rc = gemm_plan(fmt, M, N, K, v, sms, &plan);
     if (rc != W8_OK) return rc;
@@ -312,12 +313,23 @@ int w8_linear_debug(int fmt, const void* x, int ldx, const void* W_q, const floa
                          static_cast<uint8_t*>(q_out), s_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int w8_linear_resolve(int fmt, int M, int N, int K, int variant)
+{
+    int sms = 0;
+    if (check_device(&sms) != W8_OK) sms = 148;
+    GemmPlan plan;
+    const int v = resolve(fmt, M, N, K, variant, sms, &plan);
+    if (v < 0 || !(v & W8_V_FUSED)) return v;
+    const int rc = linear_plan(fmt, M, N, K, v & ~W8_V_FUSED, sms, &plan);
+    return rc == W8_OK ? v : rc;
+}
+
 size_t w8_linear_workspace_size(int fmt, int M, int N, int K, int variant)
 {
     int sms = 0;
     if (check_device(&sms) != W8_OK) sms = 148;
     GemmPlan plan;
-    if (resolve(fmt, M, N, K, variant & ~W8_V_UNFUSED, sms, &plan) < 0) return (size_t)-1;
+    if (resolve(fmt, M, N, K, variant, sms, &plan) < 0) return (size_t)-1;
     return linear_ws(plan);
 }
 

@@ -38,6 +38,22 @@ bool make_tmap(CUtensorMap* m, const void* base, int rows, int cols, int box_row
     return r == CUDA_SUCCESS;
 }
 
+// bf16 activation rows [rows, cols] with row stride ld elements, boxes of 128 elements x
+// box_rows rows, unswizzled; rows past the end read as zeros
+bool make_tmap_x(CUtensorMap* m, const void* base, int rows, int cols, int ld, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 constexpr int tile_bn(int id) { return 16 << id; }
 
 size_t stage_bytes(int bm, int bn, int kps) { return (size_t)kps * ((size_t)bm * 128 + (size_t)bn * 128); }
@@ -235,14 +251,22 @@ int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPla
         region_of(host_unit_begin(q, g), host_unit_begin(q, g + 1), q.nsb, q.kps, q.kbs, &lo, &n);
         if (n > rg) rg = n;
     }
+    // x is staged by TMA: the region's K blocks, or whole rows when per-token maxima are
+    // taken without a cluster split (then every CTA reads its rows in full)
+    const int m8 = (M + 7) & ~7;
+    const bool full_rows = fmt < W8_FMT_BLOCK_FP8 && !q.cluster;
+    const int xkb = full_rows ? q.kbs : rg;
     // the stages carry weights only; fewer of them if the region needs the room
     int st = q.stages;
-    while (st > 2 && fq_smem_bytes(q.bn, q.kps, st, rg) > 232448) --st;
-    if (fq_smem_bytes(q.bn, q.kps, st, rg) > 232448) return W8_ERR_UNSUPPORTED;
+    while (st > 2 && fq_smem_bytes(q.bn, q.kps, st, rg, m8, xkb) > 232448) --st;
+    if (fq_smem_bytes(q.bn, q.kps, st, rg, m8, xkb) > 232448) return W8_ERR_UNSUPPORTED;
     if (q.cluster && (size_t)(q.split - 1) * q.bn * q.bm * 4 > (size_t)st * q.kps * q.bm * 128) return W8_ERR_UNSUPPORTED;
     q.stages = st;
     q.rg_max_kb = rg;
-    q.smem_bytes = fq_smem_bytes(q.bn, q.kps, st, rg);
+    q.fq_m8 = m8;
+    q.fq_xkb = xkb;
+    q.fq_full_rows = full_rows ? 1 : 0;
+    q.smem_bytes = fq_smem_bytes(q.bn, q.kps, st, rg, m8, xkb);
     q.fq = 1;
     *p = q;
     return W8_OK;
@@ -254,8 +278,9 @@ int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, co
     if (!p.fq) return W8_ERR_INVALID_ARG;
     if (p.ws_bytes > 0 && (workspace == nullptr || ws_bytes < p.ws_bytes)) return W8_ERR_WORKSPACE;
     if (p.ws_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return W8_ERR_ALIGNMENT;
-    CUtensorMap tR;
+    CUtensorMap tR, tX;
     if (!make_tmap(&tR, W_q, p.rows_R, p.K, p.bm)) return W8_ERR_CUDA;
+    if (!make_tmap_x(&tX, x, p.M, p.K, ldx, p.fq_m8)) return W8_ERR_CUDA;
     GemmArgs args = {};
     args.M = p.M; args.N = p.N; args.K = p.K;
     args.swap = p.swap;
@@ -283,11 +308,14 @@ int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, co
     args.fq_block = p.fmt >= W8_FMT_BLOCK_FP8;
     args.fq_ue8m0 = p.fmt == W8_FMT_BLOCK_FP8_UE8M0;
     args.rg_max_kb = p.rg_max_kb;
+    args.fq_m8 = p.fq_m8;
+    args.fq_xkb = p.fq_xkb;
+    args.fq_full_rows = p.fq_full_rows;
     args.dbg_q = dbg_q;
     args.dbg_s = dbg_s;
     GemmMaps maps;
     maps.R = tR;
-    maps.C = tR;   // the activation map is not used: the kernel writes those tiles itself
+    maps.C = tX;   // the bf16 activation rows, staged for the in-kernel quantization
     const cudaError_t e = launch_fq(p, maps, args, s);
     if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
     return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;

@@ -90,6 +90,9 @@ struct GemmArgs {
     int fq_block;         // 1: one scale per 1 x 128 group (Block-FP8); 0: per token
     int fq_ue8m0;         // group scales as powers of two
     int rg_max_kb;        // K blocks of the largest activation region over the CTAs
+    int fq_m8;            // token rows staged from x (M rounded up to 8; rows past M are zero)
+    int fq_xkb;           // K blocks of x staged per CTA (capacity)
+    int fq_full_rows;     // stage whole rows (per-token maxima without a cluster split), else the region
     uint8_t* dbg_q;       // optional: codes of the K blocks of weight tile 0, [M, K]
     float* dbg_s;         // optional: scales, [M] or [M, K/128]
 };
@@ -111,14 +114,16 @@ __host__ __device__ inline void region_of(long long u0, long long u1, int nsb, i
     }
 }
 
-// Shared-memory bytes of the fused-quantization form: the activation region, the stages
-// (weights only), the barriers, and the per-token / per-group scale arrays.
-__host__ __device__ inline size_t fq_smem_bytes(int bn, int kps, int stages, int rg_kb)
+// Shared-memory bytes of the fused-quantization form: the activation region (codes), the
+// staged bf16 rows of x, the stages (weights only), the barriers, and the per-token /
+// per-group scale arrays.
+__host__ __device__ inline size_t fq_smem_bytes(int bn, int kps, int stages, int rg_kb, int m8, int x_kb)
 {
     const size_t region = (size_t)rg_kb * bn * 128;
-    const size_t ctrl = (size_t)(2 * stages + 2 * 2 + 5) * 8 + 16;
+    const size_t xstage = (size_t)x_kb * m8 * 256;
+    const size_t ctrl = (size_t)(2 * stages + 2 * 2 + 6) * 8 + 16;
     const size_t scal = (size_t)(4 * bn + 8 * bn + bn * rg_kb) * 4;
-    return 1024 + region + (size_t)stages * kps * 128 * 128 + ctrl + scal;
+    return 1024 + region + xstage + (size_t)stages * kps * 128 * 128 + ctrl + scal;
 }
 
 // ---------------------------------------------------------------- descriptors
@@ -304,7 +309,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = a.stages;
     uint8_t* region = smem;   // FQ: activation codes [K block][BN rows x 128 B], 128-byte swizzled
-    uint8_t* sbase = smem + (FQ ? (size_t)a.rg_max_kb * kCBytes : 0);
+    // FQ: bf16 rows of x as loaded by TMA, [K block][fq_m8 rows][128 elements]
+    uint8_t* xstage = smem + (FQ ? (size_t)a.rg_max_kb * kCBytes : 0);
+    uint8_t* sbase = xstage + (FQ ? (size_t)a.fq_xkb * a.fq_m8 * 256 : 0);
     uint64_t* full = reinterpret_cast<uint64_t*>(sbase + (size_t)S * kStageBytes);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;
@@ -314,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* red_go = red_full + 1;  // cluster split (ranks 1..): rank 0's stage memory is free
     uint64_t* a_ready = red_go + 1;   // FQ: the activation region is written
     uint64_t* amax_full = a_ready + 1;   // FQ, cluster split: the other ranks' partial row maxima landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(amax_full + 1);
+    uint64_t* x_full = amax_full + 1;    // FQ: the staged rows of x landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile int* ticket = reinterpret_cast<volatile int*>(tmem_slot + 2);
     // FQ scale arrays: per token scale, divisor (s', 1/s', factor), partial maxima of every
@@ -345,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::mbar_init(ptx::smem_u32(red_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * kEpiThreads : 1u);
         ptx::mbar_init(ptx::smem_u32(red_go), 1);
         ptx::mbar_init(ptx::smem_u32(a_ready), 1);
-        ptx::mbar_init(ptx::smem_u32(amax_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * kEpiThreads : 1u);
+        ptx::mbar_init(ptx::smem_u32(amax_full), a.csplit > 1 ? (uint32_t)(a.csplit - 1) * 32u : 1u);
+        ptx::mbar_init(ptx::smem_u32(x_full), 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -407,8 +416,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int pre = a.pdl ? (int)(n < S ? n : S) : 0;
             for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap != 0, a.swap == 0, true);
             ptx::grid_dep_wait();
-            if (!FQ)
+            if (FQ) {
+                // stage the rows of x this CTA quantizes: its region with a cluster split
+                // (the ranks together cover K), else the whole rows (their maxima need it)
+                int xlo = 0, xn = kbs;
+                if (!a.fq_full_rows) region_of(u0, u1, nsb, KPS, kbs, &xlo, &xn);
+                const uint32_t xb = ptx::smem_u32(x_full);
+                ptx::mbar_arrive_expect_tx(xb, (uint32_t)(xn * a.fq_m8 * 256));
+                for (int j = 0; j < xn; ++j)
+                    ptx::tma_load_2d(ptx::smem_u32(xstage + (size_t)j * a.fq_m8 * 256), &tmC, xb, (xlo + j) * 128, 0,
+                                     pol_a);
+            } else {
                 for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap == 0, a.swap != 0, false);
+            }
             long long issued = pre;
             int stage = pre % S;
             uint32_t phase = (pre == S) ? 1u : 0u;
@@ -514,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        if (a.pdl) {
+        if (a.pdl && !FQ) {
             // Idle until the first accumulator is ready: prefetch into L2 the weight rows
             // of the kL2Ahead units that follow the producer's first stages, so that the
             // weight stream keeps HBM busy while the kernels ahead of this one finish.
@@ -536,51 +556,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         int rg_lo = 0, rg_n = 0;
         bool fq_ok = true;
         if (FQ) {
-            // ---- fused activation quantization: row (or group) maxima, scales, then the
-            // codes of every K block this CTA multiplies, written 128-byte swizzled into the
-            // region the MMA reads in place of a TMA-loaded activation tile
+            // ---- fused activation quantization: the producer stages the bf16 rows of x
+            // by TMA; from them: row (or group) maxima, scales, then the codes of every K
+            // block this CTA multiplies, written 128-byte swizzled into the region the MMA
+            // reads in place of a TMA-loaded activation tile
             region_of(u0, u1, nsb, KPS, kbs, &rg_lo, &rg_n);
             const int te = threadIdx.x - 64;
-            const int M = a.M, K = a.K;
-            if (!a.fq_block) {
-                // per-token maxima: over this rank's K range when the cluster's ranks
-                // together cover the tile's K (cluster split), else over the whole row
-                const bool part = a.csplit > 1;
-                const int k_lo = part ? rg_lo * 128 : 0;
-                const int k_hi = part ? min((rg_lo + rg_n) * 128, K) : K;
-                const int nch = (k_hi - k_lo) >> 3;
-                const uint32_t rank = part ? ptx::cluster_ctarank() : 0u;
-                for (int m = te >> 5; m < M; m += kEpiThreads / 32) {
-                    const __nv_bfloat16* xr = a.x + (size_t)m * a.ldx + k_lo;
+            const int M = a.M, K = a.K, m8 = a.fq_m8;
+            const bool part = a.csplit > 1;
+            const uint32_t rank = part ? ptx::cluster_ctarank() : 0u;
+            const int xlo = a.fq_full_rows ? 0 : rg_lo;   // K block held by the first staged block
+            const int xn = a.fq_full_rows ? kbs : rg_n;
+            // before x arrives: zero codes for the rows past M, zero this rank's maxima
+            for (int it = te; it < (BN - M) * rg_n * 8; it += kEpiThreads) {
+                const int c16 = it & 7, kbl = (it >> 3) % rg_n, m = M + (it >> 3) / rg_n;
+                *reinterpret_cast<uint4*>(region + (size_t)kbl * kCBytes + (size_t)m * 128 + (size_t)((c16 ^ (m & 7)) << 4)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            for (int m = te; m < BN; m += kEpiThreads) amax_slots[rank * BN + m] = 0u;
+            auto xrow = [&](int kb_staged, int m) {
+                return reinterpret_cast<const uint4*>(xstage + ((size_t)kb_staged * m8 + m) * 256);
+            };
+            fq_ok = wait_bounded(ptx::smem_u32(x_full), 0, abort_flag);
+            if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !fq_ok)) fq_ok = false;
+            if (fq_ok && !a.fq_block) {
+                // per-token maxima over the staged K blocks: every epilogue thread takes
+                // 16-byte chunks of every row, then a warp maximum and a shared atomic
+                // (non-negative floats order like their bit patterns)
+                for (int m = 0; m < M; ++m) {
                     float mx = 0.0f;
-#pragma unroll 4
-                    for (int c = lane; c < nch; c += 32) {
+                    for (int c = te; c < xn * 16; c += kEpiThreads) {
                         float f[8];
-                        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(xr + (size_t)c * 8)), f);
+                        unpack_bf16x8(xrow(c >> 4, m)[c & 15], f);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(f[i]));
                     }
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-                    if (lane == 0) amax_slots[rank * BN + m] = __float_as_uint(mx);
+                    if (lane == 0 && mx > 0.0f) atomicMax(amax_slots + rank * BN + m, __float_as_uint(mx));
                 }
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
                 if (part) {
-                    // every rank sends its partial maxima to the others (distributed shared
-                    // memory) and arrives on their barriers; each thread arrives itself
-                    for (int m = te; m < M; m += kEpiThreads)
+                    // one warp per rank sends the partial maxima to the other ranks
+                    // (distributed shared memory) and arrives on their barriers
+                    if (te < 32) {
+                        for (int m = te; m < M; m += 32)
+                            for (int r = 0; r < a.csplit; ++r)
+                                if ((uint32_t)r != rank)
+                                    ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(amax_slots + rank * BN + m), (uint32_t)r),
+                                                        amax_slots[rank * BN + m]);
                         for (int r = 0; r < a.csplit; ++r)
-                            if ((uint32_t)r != rank)
-                                ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_u32(amax_slots + rank * BN + m), (uint32_t)r),
-                                                    amax_slots[rank * BN + m]);
-                    for (int r = 0; r < a.csplit; ++r)
-                        if ((uint32_t)r != rank) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(amax_full), (uint32_t)r));
+                            if ((uint32_t)r != rank) ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(amax_full), (uint32_t)r));
+                    }
                     const bool w = wait_bounded<true>(ptx::smem_u32(amax_full), 0, abort_flag);
                     if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !w)) fq_ok = false;
                 }
                 if (fq_ok) {
                     const int nslots = part ? a.csplit : 1;
-                    for (int m = te; m < BN; m += kEpiThreads) {
+                    for (int m = te; m < m8; m += kEpiThreads) {
                         float amax = 0.0f;
                         if (m < M)
                             for (int r = 0; r < nslots; ++r) amax = fmaxf(amax, __uint_as_float(amax_slots[r * BN + m]));
@@ -592,6 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         s_div[2 * BN + m] = d.f;
                         if (a.dbg_s != nullptr && blockIdx.x == 0 && m < M) a.dbg_s[m] = s;
                     }
+                    for (int m = m8 + te; m < BN; m += kEpiThreads) s_tok[m] = 1.0f;
                     ptx::bar_sync(kEpiBarrier, kEpiThreads);
                 }
             }
@@ -600,42 +634,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // of the codes)
                 const int dbg_lo = (u0 < nsb) ? (int)u0 * KPS : kbs;
                 const int dbg_hi = (u0 < nsb) ? (int)min(u1, (long long)nsb) * KPS : kbs;
-                // items: (row, K block, 16-code chunk); the 8 chunks of one row's K block
-                // are 8 consecutive lanes
-                const int total = BN * rg_n * 8;
+                // items: (token row, K block, 16-code chunk); the 8 chunks of one row's K
+                // block are 8 consecutive lanes, so a group's lanes are active together
+                const int total = M * rg_n * 8;
                 for (int it = te; it < total; it += kEpiThreads) {
                     const int c16 = it & 7;
                     const int kbl = (it >> 3) % rg_n;
                     const int m = (it >> 3) / rg_n;
                     const int kb = rg_lo + kbl;
                     const int k0 = kb * 128 + c16 * 16;
-                    const bool live = m < M && k0 < K;
                     float f[16];
-                    if (live) {
-                        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)m * a.ldx + k0);
+                    {
+                        const uint4* src = xrow(kb - xlo, m) + 2 * c16;
                         float lo[8], hi[8];
-                        unpack_bf16x8(__ldg(src), lo);
-                        unpack_bf16x8(__ldg(src + 1), hi);
+                        unpack_bf16x8(src[0], lo);
+                        unpack_bf16x8(src[1], hi);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) { f[i] = lo[i]; f[8 + i] = hi[i]; }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) f[i] = 0.0f;
                     }
                     RowDivisor d;
-                    float s = 1.0f;
                     if (a.fq_block) {
                         // one scale per 1 x 128 group: the maximum over the group's 8 lanes
+                        const unsigned gmask = 0xFFu << (lane & 24);
                         float mx = 0.0f;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) mx = fmaxf(mx, fabsf(f[i]));
 #pragma unroll
-                        for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-                        s = scale_from_amax(mx, kE4M3Max, a.fq_ue8m0 != 0);
+                        for (int o = 1; o < 8; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(gmask, mx, o));
+                        const float s = scale_from_amax(mx, kE4M3Max, a.fq_ue8m0 != 0);
                         d = make_divisor(s);
                         if (c16 == 0) s_blk[m * a.rg_max_kb + kbl] = s;
-                        if (c16 == 0 && a.dbg_s != nullptr && m < M && kb >= dbg_lo && kb < dbg_hi)
-                            a.dbg_s[(size_t)m * kbs + kb] = s;
+                        if (c16 == 0 && a.dbg_s != nullptr && kb >= dbg_lo && kb < dbg_hi) a.dbg_s[(size_t)m * kbs + kb] = s;
                     } else {
                         d.s = s_div[m];
                         d.y = s_div[BN + m];
@@ -653,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint4 codes = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                     *reinterpret_cast<uint4*>(region + (size_t)kbl * kCBytes + (size_t)m * 128 + (size_t)((c16 ^ (m & 7)) << 4)) =
                         codes;
-                    if (a.dbg_q != nullptr && live && kb >= dbg_lo && kb < dbg_hi)
+                    if (a.dbg_q != nullptr && k0 < K && kb >= dbg_lo && kb < dbg_hi)
                         *reinterpret_cast<uint4*>(a.dbg_q + (size_t)m * K + k0) = codes;
                 }
                 // the tensor core reads the region through the async proxy

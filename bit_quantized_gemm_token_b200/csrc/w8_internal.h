@@ -45,6 +45,9 @@ struct GemmPlan {
     int pfix;         // split tiles finished by all their contributors, a column slice each
     int fq;           // the kernel quantizes the activations itself (w8_linear)
     int rg_max_kb;    // fq: K blocks of the largest activation region
+    int fq_m8;        // fq: token rows staged from x (M rounded up to 8)
+    int fq_xkb;       // fq: K blocks of x staged per CTA
+    int fq_full_rows; // fq: whole rows staged (per-token maxima without a cluster split)
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile

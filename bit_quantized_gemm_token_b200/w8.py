@@ -40,7 +40,7 @@ W8_V_PDL = 1 << 16
 W8_V_CLUSTER = 1 << 17
 W8_V_BM64 = 1 << 18
 W8_V_PFIX = 1 << 19
-W8_V_UNFUSED = 1 << 24
+W8_V_FUSED = 1 << 24
 W8_V_KPS_SHIFT = 20
 W8_V_CPS_SHIFT = 22
 TILE_BN = {16: 0, 32: 1, 64: 2, 128: 3, 256: 4}
@@ -119,6 +119,8 @@ def lib():
     L.w8_linear_debug.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P, P, P]
     L.w8_linear_workspace_size.argtypes = [I, I, I, I, I]
     L.w8_linear_workspace_size.restype = S
+    L.w8_linear_resolve.argtypes = [I, I, I, I, I]
+    L.w8_linear_resolve.restype = I
     L.w8_gemm_occupancy.argtypes = [I, I, I, I, I]
     L.w8_gemm_occupancy.restype = I
     for fn in ("w8_linear", "w8_linear_debug",
@@ -330,10 +332,18 @@ def w8_linear_workspace_size(fmt, M, N, K, variant=W8_VARIANT_AUTO):
     return n
 
 
+def w8_linear_resolve(fmt, M, N, K, variant=W8_VARIANT_AUTO):
+    """The explicit variant w8_linear runs (W8_V_FUSED set for the one-kernel form)."""
+    v = lib().w8_linear_resolve(fmt, M, N, K, variant)
+    if v < 0:
+        raise W8Error("w8_linear_resolve", v)
+    return v
+
+
 def w8_linear(fmt, x, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
     """out[M, N] (bf16) = scaled quant(x) . W_q^T: x bf16 [M, K] quantized per token (or
-    per 1 x 128 group for Block-FP8) and multiplied in one call (one kernel when the
-    variant has a fused form)."""
+    per 1 x 128 group for Block-FP8) and multiplied in one call: the quantizer and the
+    GEMM, or one kernel when the variant carries W8_V_FUSED."""
     _need(x, torch.bfloat16, "x")
     M, K = x.shape
     N = W_q.shape[0]
@@ -351,7 +361,7 @@ def w8_linear(fmt, x, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace
 
 
 def w8_linear_debug(fmt, x, W_q, W_scale, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
-    """Fused w8_linear that also returns the codes [M, K] (uint8) and scales it computed."""
+    """One-kernel w8_linear that also returns the codes [M, K] (uint8) and scales it computed."""
     _need(x, torch.bfloat16, "x")
     M, K = x.shape
     N = W_q.shape[0]

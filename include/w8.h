@@ -131,7 +131,7 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 #define W8_V_CLUSTER (1 << 17)
 #define W8_V_BM64 (1 << 18)
 #define W8_V_PFIX (1 << 19)
-#define W8_V_UNFUSED (1 << 24)
+#define W8_V_FUSED (1 << 24)
 #define W8_V_KPS_SHIFT 20
 #define W8_V_CPS_SHIFT 22
 #define W8_VARIANT(swap, log2_split, tile, stream)                                            \
@@ -246,10 +246,13 @@ W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int
  *   the whole row -- and writes the codes of the K blocks it multiplies straight into
  *   shared memory, where the tensor core reads them; the quotient x / s is correctly
  *   rounded without a division per element (same codes as the quantizer kernels).
- *   Otherwise (larger M, Standard tiles) the quantizer kernel runs first into the
- *   workspace, then the GEMM.  AUTO picks the table's variant and the fused form when it
- *   exists; an explicit variant must have a fused form unless it carries W8_V_UNFUSED,
- *   which forces the two-kernel path.
+ *   Otherwise the quantizer kernel runs first into the workspace, then the GEMM (with
+ *   programmatic dependent launch when the variant asks for it).  The one-kernel form is
+ *   taken only when requested: an explicit variant carrying W8_V_FUSED (W8_ERR_UNSUPPORTED
+ *   if it has no fused form), or AUTO when the table's entry carries W8_V_FUSED.  On B200
+ *   the two-kernel chain measured faster for every decode shape: the in-kernel
+ *   quantization lengthens each CTA's path to its first MMA by more than the quantizer
+ *   kernel and its launch cost.
  * x: 16-byte aligned, ldx >= K and a multiple of 8; K as for w8_gemm.  workspace /
  * ws_bytes: at least w8_linear_workspace_size (same rules as w8_gemm's workspace; the
  * two-kernel path keeps the codes and scales there, past the 256 KiB counter area).
@@ -257,8 +260,11 @@ W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int
 W8_API int w8_linear(int fmt, const void* x, int ldx, const void* W_q, const float* W_scale, void* out, int M, int N,
                      int K, int variant, void* workspace, size_t ws_bytes, w8_stream_t stream);
 W8_API size_t w8_linear_workspace_size(int fmt, int M, int N, int K, int variant);
+/* The explicit variant w8_linear runs for this shape, with W8_V_FUSED set when it takes
+ * the one-kernel form; negative W8_ERR_* if none is legal.  Usable without a device. */
+W8_API int w8_linear_resolve(int fmt, int M, int N, int K, int variant);
 
-/* The fused form of w8_linear that also writes the codes it computed for the K blocks of
+/* The one-kernel form of w8_linear (W8_V_FUSED implied) that also writes the codes it computed for the K blocks of
  * weight tile 0 (all of K) to q_out [M, K] (16-byte aligned) and the scales to s_out
  * ([M], or [M, K/128] for Block-FP8).  For checking the fused quantization bit for bit;
  * W8_ERR_UNSUPPORTED when the variant has no fused form. */

@@ -36,7 +36,7 @@ def fused_ok(fmt, M, N, K, v):
         x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
         W = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
         sw = torch.ones(N if fmt < 2 else (N + 127) // 128 * (K // 128), device="cuda")
-        w8.w8_linear(fmt, x, W, sw, variant=v)
+        w8.w8_linear(fmt, x, W, sw, variant=v | w8.W8_V_FUSED)
         return True
     except w8.W8Error as e:
         if e.code == w8.W8_ERR_UNSUPPORTED:
@@ -82,8 +82,8 @@ def test_fused_codes_and_outputs(orc, fmt, M, N, K, vname):
     torch.cuda.synchronize()
     check_codes(orc, ofmt, x, q, s, ue8m0)
     # the same variant through the two-kernel path: identical bytes
-    two = w8.w8_linear(fmt, xd, Wd, sWd, variant=v | w8.W8_V_UNFUSED)
-    fused = w8.w8_linear(fmt, xd, Wd, sWd, variant=v)
+    two = w8.w8_linear(fmt, xd, Wd, sWd, variant=v)
+    fused = w8.w8_linear(fmt, xd, Wd, sWd, variant=v | w8.W8_V_FUSED)
     torch.cuda.synchronize()
     assert torch.equal(fused, out)
     assert torch.equal(fused, two)
@@ -118,8 +118,8 @@ def test_fused_special_rows(orc):
 
 
 def test_auto_and_two_kernel_paths(orc):
-    """AUTO takes the fused form for decode sizes and the two-kernel path otherwise (a
-    Standard tile for M = 100); both match the quantizer + GEMM calls bit for bit."""
+    """AUTO (no table entry asking for the fused form) runs the quantizer and the GEMM:
+    the same bytes as the two calls, for a Swap-AB and a Standard (M = 100) variant."""
     for M in (2, 100):
         N, K = 512, 2048
         x = synth.activations(M, K, seed=32_000 + M)
@@ -139,9 +139,9 @@ def test_explicit_variant_without_fused_form_is_rejected(orc):
     W = torch.zeros((N, K), dtype=torch.float8_e4m3fn, device="cuda")
     sw = torch.ones(N, device="cuda")
     with pytest.raises(w8.W8Error) as e:
-        w8.w8_linear(0, x, W, sw, variant=w8.variant(False, 1, 128))
+        w8.w8_linear(0, x, W, sw, variant=w8.variant(False, 1, 128) | w8.W8_V_FUSED)
     assert e.value.code == w8.W8_ERR_UNSUPPORTED
-    w8.w8_linear(0, x, W, sw, variant=w8.variant(False, 1, 128) | w8.W8_V_UNFUSED)
+    w8.w8_linear(0, x, W, sw, variant=w8.variant(False, 1, 128))
     torch.cuda.synchronize()
     assert w8.w8_device_status(clear=True) == 0
 
@@ -155,11 +155,11 @@ def test_two_kernel_path_keeps_counters_zero(orc):
     x = synth.activations(M, K, seed=33_000)
     Wq, sW = weights(orc, 0, N, K)
     Wd, sWd, xd = dev_codes(Wq, 0), dev_f32(sW), x.cuda()
-    w8.w8_linear(0, xd, Wd, sWd, variant=w8.variant(False, 1, 128) | w8.W8_V_UNFUSED, workspace=ws)
+    w8.w8_linear(0, xd, Wd, sWd, variant=w8.variant(False, 1, 128), workspace=ws)
     torch.cuda.synchronize()
     assert int(ws.buf[:65536 * 4].view(torch.int32).abs().sum()) == 0
     Aq, sA = orc.quant_rows(0, bits(x))
     _, ref, _ = orc.gemm(0, Aq, sA, Wq, sW)
-    out = w8.w8_linear(0, xd, Wd, sWd, variant=w8.variant(True, 2, 64) | w8.W8_V_UNFUSED, workspace=ws)
+    out = w8.w8_linear(0, xd, Wd, sWd, variant=w8.variant(True, 2, 64), workspace=ws)
     torch.cuda.synchronize()
     assert_bf16_close(out, ref, "split after unfused")
