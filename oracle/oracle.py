@@ -57,6 +57,7 @@ def lib():
         L.orc_silu_mul_quant_group.argtypes = [P, i, i, i, i, i, P, P]
         L.orc_silu_mul_quant_group.restype = i
         L.orc_gemm.argtypes = [i, P, P, P, P, i, i, i, i, i, P, P, P]
+        L.orc_qk_norm_rope.argtypes = [P, P, i, i, i, i, P, P, P, i, P, f]
         L.orc_gemm.restype = None
         L.orc_gemm_points.argtypes = [i, P, P, P, P, i, i, i, i, P, P, P]
         L.orc_gemm_points.restype = None
@@ -268,3 +269,18 @@ def bf16_max_err_ok(out_bits, ref_f64):
     err = np.max(np.abs(out - ref_f64)) if out.size else 0.0
     bound = 2.0 ** -7 * (np.max(np.abs(ref_f64)) if ref_f64.size else 0.0) + 1e-3
     return err <= bound, err, bound
+
+
+def qk_norm_rope(qkv_bits, Hq, Hkv, D, q_weight_bits, k_weight_bits, cos_sin, positions, eps=1e-6):
+    """Per-head rms_norm of the query / key heads of qkv_bits[T, (Hq + 2 Hkv) * D], then
+    rotate-halves rotary embedding with the fp32 table cos_sin[max_pos, D]; bf16 bits out."""
+    x = _c(qkv_bits, np.uint16)
+    T = x.shape[0]
+    out = np.zeros_like(x)
+    cs = _c(cos_sin, np.float32)
+    pos = _c(positions, np.int64)
+    rc = lib().orc_qk_norm_rope(_p(x), _p(out), T, Hq, Hkv, D, _p(_c(q_weight_bits, np.uint16)),
+                                _p(_c(k_weight_bits, np.uint16)), _p(cs), cs.shape[0], _p(pos), float(eps))
+    if rc != 0:
+        raise ValueError("orc_qk_norm_rope failed: %d" % rc)
+    return out

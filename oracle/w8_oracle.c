@@ -17,8 +17,8 @@
  *   [IT]   "Helion nel backend vLLM: un solo GEMM, tuning per forma e guadagni
  *          fino al 10%" (ai-radar.it), second and third paragraphs.
  * The pages name the operations (dynamic per-token fp8 quant, per-token-group fp8
- * quant, rms_norm + fp8 quant, silu_and_mul + fp8 quant, scaled_mm for FP8 Dynamic /
- * W8A8 INT8 / Block FP8, Split-K, Swap-AB) but print no formula.  Each function
+ * quant, rms_norm + fp8 quant, silu_and_mul + fp8 quant, fused_qk_norm_rope, scaled_mm
+ * for FP8 Dynamic / W8A8 INT8 / Block FP8, Split-K, Swap-AB) but print no formula.  Each function
  * below states the plain definition it implements; where the pages are silent the
  * comment says which reading is taken.
  *
@@ -534,5 +534,67 @@ int orc_gemm_split_k(int fmt, const uint8_t* Aq, const float* sA, const uint8_t*
         }
     }
     free(part);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* fused_qk_norm_rope                                                         */
+
+/* Per-head rms_norm of the query and key heads, then rotary position embedding ([FP8]
+ * "Kernels Helion implementados": fused_qk_norm_rope -- named there, no formula).
+ * Reading, for the merged projection qkv[T, (Hq + 2*Hkv) * D] (bf16, row-major: the Hq
+ * query heads, then the Hkv key heads, then the Hkv value heads, D values each):
+ *   for every token t and every query or key head (x = that head's D values):
+ *     y = rms_norm of x with the head-dimension weight (q_weight for query heads,
+ *         k_weight for key heads): fp64 sum of squares rounded once to fp32, then
+ *         mean = ss / D, r = 1 / sqrt(mean + eps), y_k = (x_k * r) * w_k in fp32;
+ *     with p = positions[t], c_i = cos_sin[p * D + i] and s_i = cos_sin[p * D + D/2 + i]
+ *     (i < D/2), each pair (y_i, y_{i+D/2}) is rotated by the angle whose cosine and
+ *     sine these are (the rotate-halves pairing):
+ *       o_i       = y_i * c_i - y_{i+D/2} * s_i
+ *       o_{i+D/2} = y_{i+D/2} * c_i + y_i * s_i      (fp32: two products, then the sum)
+ *     and each o is rounded once to bf16;
+ *   the value heads are copied unchanged.
+ * The cos / sin table (fp32 [max_pos, D]) is an input: the caller computes it once from
+ * the rotary base, so nothing here evaluates a transcendental function.
+ * Returns 0, or -1 for a bad size or a position outside [0, max_pos). */
+int orc_qk_norm_rope(const uint16_t* qkv, uint16_t* out, int T, int Hq, int Hkv, int D, const uint16_t* q_weight,
+                     const uint16_t* k_weight, const float* cos_sin, int max_pos, const int64_t* positions, float eps)
+{
+    if (T < 0 || Hq < 0 || Hkv < 0 || D <= 0 || D % 2 != 0) return -1;
+    const int H = Hq + 2 * Hkv;
+    const int half = D / 2;
+    float* y = (float*)malloc(sizeof(float) * (size_t)D);
+    if (!y) return -2;
+    for (int t = 0; t < T; ++t) {
+        const int64_t p = positions[t];
+        if (p < 0 || p >= max_pos) { free(y); return -1; }
+        const float* cs = cos_sin + (size_t)p * D;
+        for (int h = 0; h < H; ++h) {
+            const uint16_t* x = qkv + ((size_t)t * H + h) * D;
+            uint16_t* o = out + ((size_t)t * H + h) * D;
+            if (h >= Hq + Hkv) {
+                for (int k = 0; k < D; ++k) o[k] = x[k];
+                continue;
+            }
+            const uint16_t* w = (h < Hq) ? q_weight : k_weight;
+            double ss = 0.0;
+            for (int k = 0; k < D; ++k) {
+                double xv = (double)orc_bf16_to_float(x[k]);
+                ss += xv * xv;
+            }
+            float mean = (float)ss / (float)D;
+            float r = 1.0f / sqrtf(mean + eps);
+            for (int k = 0; k < D; ++k) y[k] = (orc_bf16_to_float(x[k]) * r) * orc_bf16_to_float(w[k]);
+            for (int i = 0; i < half; ++i) {
+                const float c = cs[i], sn = cs[half + i];
+                const float lo = y[i] * c - y[half + i] * sn;
+                const float hi = y[half + i] * c + y[i] * sn;
+                o[i] = orc_bf16_from_double((double)lo);
+                o[half + i] = orc_bf16_from_double((double)hi);
+            }
+        }
+    }
+    free(y);
     return 0;
 }
