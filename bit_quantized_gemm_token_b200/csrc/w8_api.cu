@@ -369,7 +369,27 @@ void w8_clear_table(void)
     g_table.clear();
 }
 
-int w8_device_status(int clear) { return gemm_device_status(clear); }
+int w8_device_status(int clear)
+{
+    const int g = gemm_device_status(clear);
+    const int q = qknr_device_status(clear);
+    if (g == W8_ERR_CUDA || q == W8_ERR_CUDA) return W8_ERR_CUDA;
+    return g != 0 ? g : q;
+}
+
+int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
+                    const void* k_weight, const float* cos_sin, int max_pos, const int64_t* positions, float eps,
+                    w8_stream_t stream)
+{
+    if (!qkv || !out || !q_weight || !k_weight || !cos_sin || !positions) return W8_ERR_INVALID_ARG;
+    if (T < 0 || Hq < 0 || Hkv < 0 || max_pos <= 0 || !(eps >= 0.0f)) return W8_ERR_INVALID_ARG;
+    if (D != 64 && D != 128 && D != 256) return W8_ERR_UNSUPPORTED;
+    if (!aligned(qkv, 2) || !aligned(out, 2) || !aligned(cos_sin, 4) || !aligned(positions, 8)) return W8_ERR_ALIGNMENT;
+    int rc = check_device(nullptr);
+    if (rc != W8_OK) return rc;
+    return launch_qk_norm_rope(qkv, out, T, Hq, Hkv, D, q_weight, k_weight, cos_sin, max_pos,
+                               reinterpret_cast<const long long*>(positions), eps, reinterpret_cast<cudaStream_t>(stream));
+}
 
 const char* w8_status_string(int status)
 {

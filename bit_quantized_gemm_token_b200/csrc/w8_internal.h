@@ -63,6 +63,10 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                 void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s);
 int gemm_occupancy(const GemmPlan& p, int* n);
+int launch_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
+                        const void* k_weight, const float* cos_sin, int max_pos, const long long* positions, float eps,
+                        cudaStream_t s);
+int qknr_device_status(int clear);
 // plan of the fused quantize + GEMM form of `variant`: Swap-AB with every token in one
 // narrow tile; W8_ERR_UNSUPPORTED when the variant has no such form
 int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);

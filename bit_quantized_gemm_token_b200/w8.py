@@ -116,6 +116,7 @@ def lib():
     L.w8_status_string.restype = ctypes.c_char_p
     L.w8_version.argtypes = []
     L.w8_linear.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P]
+    L.w8_qk_norm_rope.argtypes = [P, P, I, I, I, I, P, P, P, I, P, F, P]
     L.w8_linear_debug.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P, P, P]
     L.w8_linear_workspace_size.argtypes = [I, I, I, I, I]
     L.w8_linear_workspace_size.restype = S
@@ -123,7 +124,7 @@ def lib():
     L.w8_linear_resolve.restype = I
     L.w8_gemm_occupancy.argtypes = [I, I, I, I, I]
     L.w8_gemm_occupancy.restype = I
-    for fn in ("w8_linear", "w8_linear_debug",
+    for fn in ("w8_linear", "w8_linear_debug", "w8_qk_norm_rope",
                "w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant",
                "w8_rmsnorm_quant_group", "w8_silu_mul_quant_group", "w8_gemm",
                "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
@@ -322,6 +323,26 @@ def w8_gemm(fmt, A_q, A_scale, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, 
     rc = lib().w8_gemm(fmt, _ptr(A_q), _ptr(A_scale), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp, wn,
                        _stream(stream))
     _check("w8_gemm", rc)
+    return out
+
+
+def w8_qk_norm_rope(qkv, Hq, Hkv, D, q_weight, k_weight, cos_sin, positions, eps=1e-6, out=None, stream=None):
+    """Query/key per-head rms_norm + rotary embedding of qkv [T, (Hq + 2 Hkv) * D] bf16;
+    out=qkv works in place.  cos_sin fp32 [max_pos, D]; positions int64 [T]."""
+    _need(qkv, torch.bfloat16, "qkv")
+    T = qkv.shape[0]
+    if qkv.shape[1] != (Hq + 2 * Hkv) * D or not qkv.is_contiguous():
+        raise ValueError("qkv must be contiguous [T, (Hq + 2 Hkv) * D]")
+    if out is None:
+        out = torch.empty_like(qkv)
+    _need(out, torch.bfloat16, "out")
+    _need(q_weight, torch.bfloat16, "q_weight")
+    _need(k_weight, torch.bfloat16, "k_weight")
+    _need(cos_sin, torch.float32, "cos_sin")
+    _need(positions, torch.int64, "positions")
+    rc = lib().w8_qk_norm_rope(_ptr(qkv), _ptr(out), T, Hq, Hkv, D, _ptr(q_weight), _ptr(k_weight), _ptr(cos_sin),
+                               cos_sin.shape[0], _ptr(positions), float(eps), _stream(stream))
+    _check("w8_qk_norm_rope", rc)
     return out
 
 

@@ -233,6 +233,26 @@ W8_API int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant);
 W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int N, int K, int variant,
                       void* workspace, size_t ws_bytes, w8_stream_t stream);
 
+/* Query/key rms_norm + rotary embedding on the merged attention projection ("PyTorch
+ * integra Helion en vLLM para acelerar inferencia FP8", section "Kernels Helion
+ * implementados": fused_qk_norm_rope; named there without a formula).  Reading:
+ *   qkv, out  bf16 [T, (Hq + 2*Hkv) * D] row-major: Hq query heads, Hkv key heads, Hkv
+ *             value heads, D contiguous values each; out may equal qkv (in place);
+ *   for each token t and query (key) head: y = rms_norm(head) with q_weight (k_weight)
+ *             [D] bf16 -- sum of squares in fp64 rounded once to fp32, r = 1/sqrt(ss/D
+ *             + eps), y_k = (x_k * r) * w_k in fp32 -- then each pair (y_i, y_{i+D/2}) is
+ *             rotated by the angle of position p = positions[t]: o_i = y_i c_i -
+ *             y_{i+D/2} s_i, o_{i+D/2} = y_{i+D/2} c_i + y_i s_i, c_i = cos_sin[p*D + i],
+ *             s_i = cos_sin[p*D + D/2 + i] (fp32 table [max_pos, D], the caller's);
+ *             rounded to bf16.  Value heads are copied unchanged.
+ *   positions int64 [T] in [0, max_pos): a position outside records W8_ERR_INVALID_ARG
+ *             in the device status word (w8_device_status) and leaves that token's
+ *             query and key heads unwritten.
+ * D must be 64, 128 or 256 (W8_ERR_UNSUPPORTED otherwise). */
+W8_API int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
+                           const void* k_weight, const float* cos_sin, int max_pos, const int64_t* positions,
+                           float eps, w8_stream_t stream);
+
 /* Quantize-and-multiply in one call: out = w8_gemm(fmt, quant(x), W) for a bf16
  * activation x [M, K] (row stride ldx elements), with quant the per-token quantizer of
  * w8_quant_per_token for FP8-dynamic (e4m3) and W8A8-INT8 (int8), or its 1 x 128 group
