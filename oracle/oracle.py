@@ -284,3 +284,29 @@ def qk_norm_rope(qkv_bits, Hq, Hkv, D, q_weight_bits, k_weight_bits, cos_sin, po
     if rc != 0:
         raise ValueError("orc_qk_norm_rope failed: %d" % rc)
     return out
+
+
+def grouped_gemm(fmt, Aq, sA, Wq, sW, offsets):
+    """Grouped (mixture-of-experts) scaled GEMM: the activations' rows are sorted by
+    expert, rows [offsets[e], offsets[e+1]) belong to expert e, and each is multiplied
+    by that expert's weights Wq[e] [N, K] with its per-channel scales sW[e] [N]
+    (FP8-dynamic, fmt 0, or W8A8-INT8, fmt 1): the plain GEMM of this module, expert by
+    expert.  Returns (out_bf16_bits[T, N], ref_f64[T, N], acc_i64 or None)."""
+    Aq = np.asarray(Aq)
+    off = np.asarray(offsets, dtype=np.int64)
+    E, N, K = np.asarray(Wq).shape
+    T = Aq.shape[0]
+    if off.shape != (E + 1,) or off[0] != 0 or off[-1] > T or np.any(np.diff(off) < 0):
+        raise ValueError("offsets must rise from 0 to at most T")
+    out = np.zeros((T, N), dtype=np.uint16)
+    ref = np.zeros((T, N), dtype=np.float64)
+    acc = np.zeros((T, N), dtype=np.int64) if fmt == 1 else None
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi == lo:
+            continue
+        o, r, a = gemm(fmt, Aq[lo:hi], np.asarray(sA)[lo:hi], np.asarray(Wq)[e], np.asarray(sW)[e])
+        out[lo:hi], ref[lo:hi] = o, r
+        if acc is not None:
+            acc[lo:hi] = a
+    return out, ref, acc
