@@ -66,6 +66,14 @@ namespace {
 // Built-in rule when the table has no entry: Swap-AB with the narrowest token tile for
 // decode-sized M, the Standard 128 x 128 tile otherwise; always the balanced partition
 // (weights are streamed evenly by every SM; the partial-sum traffic stays in L2).
+// Grouped GEMM default: Swap-AB over the balanced partition with the narrowest token tile
+// that holds an expert's largest token count (64 beyond that: several token tiles).
+int grouped_variant(int max_m)
+{
+    const int tile = max_m <= 16 ? kTileBN16 : max_m <= 32 ? kTileBN32 : kTileBN64;
+    return W8_VARIANT(1, 0, tile, 1);
+}
+
 int builtin_variant(int fmt, int M)
 {
     const bool block = fmt >= W8_FMT_BLOCK_FP8;
@@ -375,6 +383,37 @@ int w8_device_status(int clear)
     const int q = qknr_device_status(clear);
     if (g == W8_ERR_CUDA || q == W8_ERR_CUDA) return W8_ERR_CUDA;
     return g != 0 ? g : q;
+}
+
+int w8_grouped_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale, void* out,
+                    const int* expert_offsets, int E, int T, int N, int K, int max_tokens_per_expert, int variant,
+                    void* workspace, size_t ws_bytes, w8_stream_t stream)
+{
+    if (!A_q || !A_scale || !W_q || !W_scale || !out || !expert_offsets) return W8_ERR_INVALID_ARG;
+    if (E <= 0 || T <= 0 || N <= 0 || K <= 0 || max_tokens_per_expert <= 0) return W8_ERR_INVALID_ARG;
+    if (!aligned(A_q, 16) || !aligned(W_q, 16) || !aligned(out, 2) || !aligned(expert_offsets, 4)) return W8_ERR_ALIGNMENT;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != W8_OK) return rc;
+    const int mm = max_tokens_per_expert < T ? max_tokens_per_expert : T;
+    const int v = (variant & W8_V_EXPLICIT) ? variant : (grouped_variant(mm) | (variant & W8_V_PDL));
+    GemmPlan plan;
+    rc = grouped_plan(fmt, T, N, K, E, mm, v, sms, &plan);
+    if (rc != W8_OK) return rc;
+    return gemm_launch(plan, A_q, A_scale, W_q, W_scale, out, nullptr, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), expert_offsets);
+}
+
+size_t w8_grouped_gemm_workspace_size(int fmt, int E, int T, int N, int K, int max_tokens_per_expert, int variant)
+{
+    int sms = 0;
+    if (check_device(&sms) != W8_OK) sms = 148;
+    if (T <= 0 || max_tokens_per_expert <= 0) return (size_t)-1;
+    const int mm = max_tokens_per_expert < T ? max_tokens_per_expert : T;
+    const int v = (variant & W8_V_EXPLICIT) ? variant : (grouped_variant(mm) | (variant & W8_V_PDL));
+    GemmPlan plan;
+    if (grouped_plan(fmt, T, N, K, E, mm, v, sms, &plan) != W8_OK) return (size_t)-1;
+    return plan.ws_bytes;
 }
 
 int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,

@@ -183,14 +183,15 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
 
 // ---------------------------------------------------------------- launch
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
-                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s)
+                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s, const int* g_off)
 {
     if (p.ws_bytes > 0 && (workspace == nullptr || ws_bytes < p.ws_bytes)) return W8_ERR_WORKSPACE;
     if (p.ws_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return W8_ERR_ALIGNMENT;
     CUtensorMap tR, tC;
     const void* R = p.swap ? W_q : A_q;
     const void* C = p.swap ? A_q : W_q;
-    if (!make_tmap(&tR, R, p.rows_R, p.K, p.bm)) return W8_ERR_CUDA;
+    // the grouped form's weights are the experts' [N, K] matrices one after another
+    if (!make_tmap(&tR, R, p.grouped ? p.rows_R * p.g_E : p.rows_R, p.K, p.bm)) return W8_ERR_CUDA;
     if (!make_tmap(&tC, C, p.rows_C, p.K, p.bn)) return W8_ERR_CUDA;
 
     GemmArgs args = {};
@@ -205,6 +206,9 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     args.align_tiles = p.align_tiles;
     args.csplit = p.cluster ? p.split : 0;
     args.pfix = p.pfix;
+    args.grouped = p.grouped;
+    args.g_E = p.g_E;
+    args.g_off = g_off;
     args.w_ptr = static_cast<const uint8_t*>(W_q);
     args.stages = p.stages;
     args.pdl = p.pdl;
@@ -268,6 +272,36 @@ int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPla
     q.fq_full_rows = full_rows ? 1 : 0;
     q.smem_bytes = fq_smem_bytes(q.bn, q.kps, st, rg, m8, xkb);
     q.fq = 1;
+    *p = q;
+    return W8_OK;
+}
+
+int grouped_plan(int fmt, int T, int N, int K, int E, int max_m, int variant, int sm_count, GemmPlan* p)
+{
+    if (E <= 0 || max_m <= 0 || max_m > T) return W8_ERR_INVALID_ARG;
+    if (fmt != W8_FMT_FP8_DYN && fmt != W8_FMT_INT8) return W8_ERR_UNSUPPORTED;
+    GemmPlan q;
+    // the shape of one expert's GEMM at its largest token count fixes the tiles
+    int rc = gemm_plan(fmt, max_m, N, K, variant, sm_count, &q);
+    if (rc != W8_OK) return rc;
+    // Swap-AB, balanced partition over the SMs, reductions through the workspace
+    if (!q.swap || !q.stream || q.cluster || q.pfix || q.bm != 128) return W8_ERR_UNSUPPORTED;
+    const long long tiles_max = (long long)E * q.r_tiles * q.c_tiles;
+    if (tiles_max > kMaxCounterTiles) return W8_ERR_UNSUPPORTED;
+    q.grouped = 1;
+    q.g_E = E;
+    q.M = T;
+    q.rows_C = T;
+    // one CTA per SM (or the variant's CTAs per SM): the units are counted on the device
+    const int cps = ((variant >> W8_V_CPS_SHIFT) & 0x3) ? ((variant >> W8_V_CPS_SHIFT) & 0x3) : 1;
+    q.G = (sm_count > 0 ? sm_count : 148) * cps;
+    // tile counts and offsets of the experts, kept in shared memory
+    q.smem_bytes += (size_t)(2 * (E + 1)) * 4 + 16;
+    if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
+    // the balanced partition deals out the units of the experts that have tokens; the
+    // partial slots are per CTA and the counter area has its fixed size
+    q.ws_counters = (size_t)kMaxCounterTiles * 4;
+    q.ws_bytes = q.ws_counters + (size_t)q.G * 2 * (size_t)q.bn * q.bm * 4;
     *p = q;
     return W8_OK;
 }

@@ -93,6 +93,11 @@ struct GemmArgs {
     int fq_m8;            // token rows staged from x (M rounded up to 8; rows past M are zero)
     int fq_xkb;           // K blocks of x staged per CTA (capacity)
     int fq_full_rows;     // stage whole rows (per-token maxima without a cluster split), else the region
+    // grouped (mixture-of-experts) form: tokens sorted by expert, rows [g_off[e],
+    // g_off[e+1]) of A belong to expert e, whose weights are rows [e N, (e+1) N) of W
+    int grouped;
+    int g_E;
+    const int* g_off;     // device [g_E + 1]
     uint8_t* dbg_q;       // optional: codes of the K blocks of weight tile 0, [M, K]
     float* dbg_s;         // optional: scales, [M] or [M, K/128]
 };
@@ -153,15 +158,17 @@ __device__ __forceinline__ constexpr uint32_t instr_desc()
 }
 
 // ---------------------------------------------------------------- unit partition
-__device__ __forceinline__ long long unit_begin(const GemmArgs& a, long long g)
+// U = total units and G = CTAs sharing them (a.units and a.G, or counted on the device
+// in the grouped form, where CTAs past the unit count get nothing)
+__device__ __forceinline__ long long unit_begin(const GemmArgs& a, long long g, long long U, long long G)
 {
     if (a.align_tiles) return (g * a.tiles / a.G) * a.nsb;
-    return g * a.units / a.G;
+    return g * U / G;
 }
 
-__device__ __forceinline__ int cta_of_unit(const GemmArgs& a, long long u)
+__device__ __forceinline__ int cta_of_unit(const GemmArgs& a, long long u, long long U, long long G)
 {
-    return (int)(((u + 1) * (long long)a.G - 1) / a.units);
+    return (int)(((u + 1) * G - 1) / U);
 }
 
 // ---------------------------------------------------------------- bounded waits
@@ -228,13 +235,16 @@ __device__ __forceinline__ uint32_t add_words(uint32_t x, uint32_t y)
 
 // Store one output element (row i of the R tile, column j of the C tile).  `w` is the
 // raw accumulator word: unscaled (FP8/INT8) or already block-scaled (BLOCK).
+// Swap-AB: [m_lo, m_hi) bounds the output rows (tokens, the C side) a tile may write --
+// its own tokens; in the grouped form the neighbouring rows belong to other experts
 template <int KIND, bool BLOCK>
 __device__ __forceinline__ void store_out(const GemmArgs& a, const float* tokscale, int r_row, int c_row, uint32_t w,
-                                          float s_row)
+                                          float s_row, int m_lo = 0, int m_hi = 0x7FFFFFFF)
 {
     const int m = a.swap ? c_row : r_row;
     const int n = a.swap ? r_row : c_row;
     if (m >= a.M || n >= a.N) return;
+    if (a.swap && (m < m_lo || m >= m_hi)) return;
     const size_t o = (size_t)m * a.N + n;
     if (KIND == KIND_I8 && a.out_i32 != nullptr) {
         a.out_i32[o] = (int32_t)w;
@@ -260,7 +270,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 // Standard form these are 16 consecutive outputs of one row: two 16-byte stores.
 template <int KIND, bool BLOCK>
 __device__ __forceinline__ void store_chunk16(const GemmArgs& a, const float* tokscale, int r_row, int c_base,
-                                              const uint32_t (&v)[16], float s_row)
+                                              const uint32_t (&v)[16], float s_row, int m_lo = 0, int m_hi = 0x7FFFFFFF)
 {
     if (!a.swap && a.vec_ok && a.out_i32 == nullptr && r_row < a.M && c_base + 15 < a.N) {
         float f[16];
@@ -280,7 +290,7 @@ __device__ __forceinline__ void store_chunk16(const GemmArgs& a, const float* to
         return;
     }
 #pragma unroll
-    for (int jj = 0; jj < 16; ++jj) store_out<KIND, BLOCK>(a, tokscale, r_row, c_base + jj, v[jj], s_row);
+    for (int jj = 0; jj < 16; ++jj) store_out<KIND, BLOCK>(a, tokscale, r_row, c_base + jj, v[jj], s_row, m_lo, m_hi);
 }
 
 __device__ __forceinline__ bool first_epi_thread(unsigned t) { return t == 64; }
@@ -384,10 +394,92 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem = *tmem_slot;
     }
 
-    const long long u0 = unit_begin(a, blockIdx.x);
-    const long long u1 = unit_begin(a, blockIdx.x + 1);
     const int nsb = a.nsb;   // stage blocks per tile
     const int kbs = a.kbs;   // 128-column K blocks per tile
+    // grouped form: per-expert tile counts from the expert offsets (written by the kernels
+    // ahead, hence after the wait), as prefix sums in shared memory; every CTA derives the
+    // same balanced partition of the units of the experts that have tokens
+    int* s_gtile = reinterpret_cast<int*>(tmem_slot + 4);     // [g_E + 1] tile prefix
+    int* s_goff = s_gtile + (a.grouped ? a.g_E + 1 : 0);       // [g_E + 1] clamped offsets
+    long long U = a.units;
+    if (a.grouped) {
+        ptx::grid_dep_wait();
+        if (warp == 0) {
+            const int E = a.g_E, T = a.rows_C;
+            const int per = (E + 31) / 32;
+            const int e0 = lane * per, e1 = min(e0 + per, E);
+            // offsets must rise within [0, T]; otherwise nothing is computed and the
+            // device status records W8_ERR_INVALID_ARG
+            bool bad = false;
+            for (int e = e0; e < e1; ++e) {
+                const int lo = a.g_off[e], hi = a.g_off[e + 1];
+                bad |= lo < 0 || hi > T || hi < lo;
+            }
+            const bool any_bad = __any_sync(0xFFFFFFFFu, bad);
+            int tiles = 0;
+            for (int e = e0; e < e1; ++e) {
+                const int lo = any_bad ? 0 : a.g_off[e], hi = any_bad ? 0 : a.g_off[e + 1];
+                s_goff[e] = lo;
+                if (e == E - 1) s_goff[E] = hi;
+                tiles += a.r_tiles * ((hi - lo + BN - 1) / BN);
+            }
+            // exclusive scan of the lanes' tile counts
+            int incl = tiles;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int run = incl - tiles;
+            for (int e = e0; e < e1; ++e) {
+                s_gtile[e] = run;
+                const int lo = any_bad ? 0 : a.g_off[e], hi = any_bad ? 0 : a.g_off[e + 1];
+                run += a.r_tiles * ((hi - lo + BN - 1) / BN);
+            }
+            if (lane == 31) s_gtile[E] = incl;
+            if (any_bad && lane == 0) record_error(W8_ERR_INVALID_ARG);
+        }
+        __syncthreads();
+        U = (long long)s_gtile[a.g_E] * nsb;
+    }
+    // every CTA of the partition must own at least one unit (a split tile is finished by
+    // its contributors, consecutive CTAs): with fewer units than CTAs the rest idle
+    const long long Gp = (a.grouped && U < a.G) ? U : a.G;
+    const long long u0 = ((long long)blockIdx.x < Gp) ? unit_begin(a, blockIdx.x, U, Gp) : U;
+    const long long u1 = ((long long)blockIdx.x < Gp) ? unit_begin(a, blockIdx.x + 1, U, Gp) : U;
+    // tile t -> weight tile rt, token tile ct, the rows they start at in W and A, and the
+    // number of valid rows on the C side (tokens of the expert, in the grouped form).
+    // Grouped: the token box starts at c_off + ct * BN unless that would run it past the
+    // last token row; then it starts earlier (at row T - BN, or 0) and the tile's tokens
+    // sit c_shift columns into it.
+    auto tile_loc = [&](int t, int& rt, int& ct, int& r_off, int& c_off, int& c_valid, int& c_shift) {
+        c_shift = 0;
+        if (!a.grouped) {
+            rt = t / a.c_tiles;
+            ct = t % a.c_tiles;
+            r_off = 0;
+            c_off = 0;
+            c_valid = a.rows_C;
+            return;
+        }
+        // the expert e with s_gtile[e] <= t < s_gtile[e + 1] (it has tiles)
+        int lo = 0, hi = a.g_E;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_gtile[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int m_e = s_goff[lo + 1] - s_goff[lo];
+        const int ctiles = (m_e + BN - 1) / BN;
+        const int lt = t - s_gtile[lo];
+        rt = lt / ctiles;
+        ct = lt % ctiles;
+        r_off = lo * a.rows_R;
+        const int start = s_goff[lo] + ct * BN;
+        const int box = min(start, max(0, a.rows_C - BN));
+        c_shift = start - box;
+        c_off = box - ct * BN;    // so that c_off + ct * BN is the box's first row
+        c_valid = min(m_e, ct * BN + (BN - c_shift));   // tokens of this tile end by column BN
+    };
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -401,19 +493,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue = [&](int s, long long u, bool load_r, bool load_c, bool expect) {
                 const int t = (int)(u / nsb), kb0 = (int)(u % nsb) * KPS;
                 const int nkb = (kbs - kb0 < KPS) ? kbs - kb0 : KPS;
-                const int rt = t / a.c_tiles, ct = t % a.c_tiles;
+                int rt, ct, r_off, c_off, c_valid, c_shift;
+                tile_loc(t, rt, ct, r_off, c_off, c_valid, c_shift);
                 const uint32_t fb = ptx::smem_u32(full + s);
                 if (expect) ptx::mbar_arrive_expect_tx(fb, (uint32_t)(nkb * (kRBytes + (FQ ? 0 : kCBytes))));
                 for (int j = 0; j < nkb; ++j) {
-                    if (load_r) ptx::tma_load_2d(ptx::smem_u32(r_slot(s, j)), &tmR, fb, (kb0 + j) * 128, rt * BM, pol_R);
-                    if (load_c && !FQ) ptx::tma_load_2d(ptx::smem_u32(c_slot(s, j)), &tmC, fb, (kb0 + j) * 128, ct * BN, pol_C);
+                    if (load_r) ptx::tma_load_2d(ptx::smem_u32(r_slot(s, j)), &tmR, fb, (kb0 + j) * 128, r_off + rt * BM, pol_R);
+                    if (load_c && !FQ) ptx::tma_load_2d(ptx::smem_u32(c_slot(s, j)), &tmC, fb, (kb0 + j) * 128, c_off + ct * BN, pol_C);
                 }
             };
             // With programmatic dependent launch, before waiting for the kernels ahead of
             // this one, the producer requests the weight boxes of the first `pre` stages
             // (weights are never the output of work in flight; the epilogue warps prefetch
             // the next units' weights into L2); the activation boxes follow after the wait.
-            const int pre = a.pdl ? (int)(n < S ? n : S) : 0;
+            const int pre = (a.pdl && !a.grouped) ? (int)(n < S ? n : S) : 0;
             for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap != 0, a.swap == 0, true);
             ptx::grid_dep_wait();
             if (FQ) {
@@ -534,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        if (a.pdl && !FQ) {
+        if (a.pdl && !FQ && !a.grouped) {
             // Idle until the first accumulator is ready: prefetch into L2 the weight rows
             // of the kL2Ahead units that follow the producer's first stages, so that the
             // weight stream keeps HBM busy while the kernels ahead of this one finish.
@@ -710,7 +803,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int sb_lo = (int)(u % nsb);
             const long long rem = u1 - u;
             const int sb_hi = (int)((nsb - sb_lo < rem) ? nsb : sb_lo + rem);
-            const int rt = t / a.c_tiles, ct = t % a.c_tiles;
+            int rt, ct, r_off, c_off, c_valid, c_shift;
+            tile_loc(t, rt, ct, r_off, c_off, c_valid, c_shift);
             // sentinel for threads holding no real row: padding lanes of the 64-row tile and,
             // in the Standard form, token rows past M (their accumulators are zero)
             const int r_row = (lane_has_row && rt * BM + i < a.rows_R) ? rt * BM + i : 0x7FFFFFFF;
@@ -719,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot = (u == u0) ? 0 : 1;
             // scale of this thread's R-side index (FP8 / INT8; BLOCK scales per K block)
             float s_row = 1.0f;
-            if (!BLOCK && a.out_i32 == nullptr && r_row < a.rows_R) s_row = __ldg((a.swap ? a.sW : a.sA) + r_row);
+            if (!BLOCK && a.out_i32 == nullptr && r_row < a.rows_R) s_row = __ldg((a.swap ? a.sW : a.sA) + r_off + r_row);
 
             float acc[kAccRegs];
 #pragma unroll
@@ -785,7 +879,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // columns of this tile that hold real rows of the C operand (tokens for
             // Swap-AB: only these are written, published and reduced)
-            const int ncv = (a.rows_C - ct * BN < BN) ? a.rows_C - ct * BN : BN;
+            // columns [c_shift, ncv) of the tile are its tokens (c_shift > 0 only in the
+            // grouped form, where the box may start before the tile's first token)
+            const int ncv = c_shift + ((c_valid - ct * BN < BN - c_shift) ? c_valid - ct * BN : BN - c_shift);
+            const int c_base = c_off + ct * BN;   // first output row (Swap-AB) / column of this tile
+            const int m_lo = c_base + c_shift;    // first token this tile may write
+            const int m_hi = c_base + ncv;        // one past its last
             // 64-row token tile: only nrows rows are real tokens; its partials are kept as
             // [row][column] and reduced column-parallel by all 128 epilogue threads
             constexpr bool kCompact = (BM == 64);
@@ -896,7 +995,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int jj = 0; jj < 16; ++jj)
                                 v[jj] = add_words<BLOCK ? KIND_F8 : KIND>(v[jj], src[(c0 + jj) * BM + i]);
                         }
-                        store_chunk16<KIND, BLOCK>(a, tokscale, r_row, ct * BN + c0, v, s_row);
+                        store_chunk16<KIND, BLOCK>(a, tokscale, r_row, c_base + c0, v, s_row, m_lo, m_hi);
                     }
                 }
             } else if (full_tile) {
@@ -906,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (c0 >= ncv) break;
                     uint32_t v[16];
                     fetch16(c0, v);
-                    store_chunk16<KIND, BLOCK>(a, tokscale, r_row, ct * BN + c0, v, s_row);
+                    store_chunk16<KIND, BLOCK>(a, tokscale, r_row, c_base + c0, v, s_row, m_lo, m_hi);
                 }
             } else {
                 // ---- partial: publish to this CTA's slot ([column][row] words, coalesced)
@@ -940,8 +1039,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
                 if (first_epi) *ticket = atomicAdd(a.counters + t, 1);
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
-                const int g_lo = cta_of_unit(a, (long long)t * nsb);
-                const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1);
+                const int g_lo = cta_of_unit(a, (long long)t * nsb, U, Gp);
+                const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1, U, Gp);
                 if (*ticket == g_hi - g_lo && kCompact) {
                     // column-parallel: per column and row, contributors added in CTA order,
                     // four contributors' loads in flight together
@@ -960,7 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     const int c = g_lo + cb + k;
                                     const uint32_t* p = nullptr;
                                     if (cb + k < nc) {
-                                        const int sl = (unit_begin(a, c) / nsb == t) ? 0 : 1;
+                                        const int sl = (unit_begin(a, c, U, Gp) / nsb == t) ? 0 : 1;
                                         p = a.partials + ((size_t)c * 2 + sl) * (size_t)(BN * BM) + col;
                                     }
 #pragma unroll
@@ -996,7 +1095,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int k = 0; k < 4; ++k) {
                                 const int c = g_lo + cb + k;
                                 if (cb + k < nc) {
-                                    const int sl = (unit_begin(a, c) / nsb == t) ? 0 : 1;
+                                    const int sl = (unit_begin(a, c, U, Gp) / nsb == t) ? 0 : 1;
                                     const uint32_t* p = a.partials + ((size_t)c * 2 + sl) * (size_t)(BN * BM);
 #pragma unroll
                                     for (int jj = 0; jj < 16; ++jj)
@@ -1012,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 }
                             }
                         }
-                        store_chunk16<KIND, BLOCK>(a, tokscale, r_row, ct * BN + c0, v, s_row);
+                        store_chunk16<KIND, BLOCK>(a, tokscale, r_row, c_base + c0, v, s_row, m_lo, m_hi);
                     }
                     if (first_epi) a.counters[t] = 0;   // leave the counter ready for the next call
                 }
@@ -1029,8 +1128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int f = 0; f < nfix && f < 2; ++f) {
                 const int t = fix_t[f];
                 const int rt = t / a.c_tiles, ct = t % a.c_tiles;
-                const int g_lo = cta_of_unit(a, (long long)t * nsb);
-                const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1);
+                const int g_lo = cta_of_unit(a, (long long)t * nsb, U, Gp);
+                const int g_hi = cta_of_unit(a, (long long)t * nsb + nsb - 1, U, Gp);
                 const int nc = g_hi - g_lo + 1;
                 const int j = (int)blockIdx.x - g_lo;
                 bool w = true;
@@ -1049,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < 8; ++k) {
                             const int c = g_lo + cb + k;
                             if (cb + k < nc) {
-                                const int sl = (unit_begin(a, c) / nsb == t) ? 0 : 1;
+                                const int sl = (unit_begin(a, c, U, Gp) / nsb == t) ? 0 : 1;
                                 const uint32_t* p = a.partials + ((size_t)c * 2 + sl) * (size_t)(BN * BM) +
                                                     (size_t)r * BN + 4 * cg;
                                 x[k] = __ldcg(reinterpret_cast<const uint4*>(p));

@@ -48,6 +48,8 @@ struct GemmPlan {
     int fq_m8;        // fq: token rows staged from x (M rounded up to 8)
     int fq_xkb;       // fq: K blocks of x staged per CTA
     int fq_full_rows; // fq: whole rows staged (per-token maxima without a cluster split)
+    int grouped;      // mixture-of-experts form: M = all tokens, N per expert
+    int g_E;          // grouped: experts
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile
@@ -61,7 +63,8 @@ struct GemmPlan {
 
 int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
-                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s);
+                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s,
+                const int* g_off = nullptr);
 int gemm_occupancy(const GemmPlan& p, int* n);
 int launch_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
                         const void* k_weight, const float* cos_sin, int max_pos, const long long* positions, float eps,
@@ -70,6 +73,9 @@ int qknr_device_status(int clear);
 // plan of the fused quantize + GEMM form of `variant`: Swap-AB with every token in one
 // narrow tile; W8_ERR_UNSUPPORTED when the variant has no such form
 int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);
+// plan of the grouped (mixture-of-experts) GEMM: T tokens sorted by expert, E experts of
+// N x K weights, at most max_m tokens per expert (sizes the token tiles and counters)
+int grouped_plan(int fmt, int T, int N, int K, int E, int max_m, int variant, int sm_count, GemmPlan* p);
 // fused launch: x bf16 [M, K] (row stride ldx) is quantized inside the GEMM kernel;
 // dbg_q / dbg_s (optional) receive the codes and scales of weight tile 0's K blocks
 int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, const float* W_scale, void* out,

@@ -117,6 +117,9 @@ def lib():
     L.w8_version.argtypes = []
     L.w8_linear.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P]
     L.w8_qk_norm_rope.argtypes = [P, P, I, I, I, I, P, P, P, I, P, F, P]
+    L.w8_grouped_gemm.argtypes = [I, P, P, P, P, P, P, I, I, I, I, I, I, P, S, P]
+    L.w8_grouped_gemm_workspace_size.argtypes = [I, I, I, I, I, I, I]
+    L.w8_grouped_gemm_workspace_size.restype = S
     L.w8_linear_debug.argtypes = [I, P, I, P, P, P, I, I, I, I, P, S, P, P, P]
     L.w8_linear_workspace_size.argtypes = [I, I, I, I, I]
     L.w8_linear_workspace_size.restype = S
@@ -124,7 +127,7 @@ def lib():
     L.w8_linear_resolve.restype = I
     L.w8_gemm_occupancy.argtypes = [I, I, I, I, I]
     L.w8_gemm_occupancy.restype = I
-    for fn in ("w8_linear", "w8_linear_debug", "w8_qk_norm_rope",
+    for fn in ("w8_linear", "w8_linear_debug", "w8_qk_norm_rope", "w8_grouped_gemm",
                "w8_quant_per_token", "w8_quant_weight_block", "w8_rmsnorm_quant", "w8_silu_mul_quant",
                "w8_rmsnorm_quant_group", "w8_silu_mul_quant_group", "w8_gemm",
                "w8_gemm_resolve_variant", "w8_gemm_i32_debug", "w8_load_table", "w8_device_status", "w8_version"):
@@ -323,6 +326,36 @@ def w8_gemm(fmt, A_q, A_scale, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, 
     rc = lib().w8_gemm(fmt, _ptr(A_q), _ptr(A_scale), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp, wn,
                        _stream(stream))
     _check("w8_gemm", rc)
+    return out
+
+
+def w8_grouped_gemm_workspace_size(fmt, E, T, N, K, max_tokens_per_expert, variant=W8_VARIANT_AUTO):
+    n = lib().w8_grouped_gemm_workspace_size(fmt, E, T, N, K, max_tokens_per_expert, variant)
+    if n == ctypes.c_size_t(-1).value:
+        raise W8Error("w8_grouped_gemm_workspace_size", W8_ERR_INVALID_ARG)
+    return n
+
+
+def w8_grouped_gemm(fmt, A_q, A_scale, W_q, W_scale, expert_offsets, max_tokens_per_expert=None, out=None,
+                    variant=W8_VARIANT_AUTO, workspace=None, stream=None):
+    """Mixture-of-experts GEMM: A_q [T, K] rows sorted by expert (rows [off[e], off[e+1])
+    belong to expert e), W_q [E, N, K], W_scale [E, N]; expert_offsets int32 [E+1] on the
+    device.  Rows no expert owns are left as they were in `out`."""
+    T, K = A_q.shape
+    E, N, K2 = W_q.shape
+    if K2 != K:
+        raise ValueError("K mismatch")
+    if expert_offsets.dtype != torch.int32 or not expert_offsets.is_cuda or expert_offsets.numel() != E + 1:
+        raise TypeError("expert_offsets must be a CUDA int32 tensor of E + 1 entries")
+    mm = T if max_tokens_per_expert is None else int(max_tokens_per_expert)
+    if out is None:
+        out = torch.zeros((T, N), dtype=torch.bfloat16, device=A_q.device)
+    _need(out, torch.bfloat16, "out")
+    nbytes = w8_grouped_gemm_workspace_size(fmt, E, T, N, K, mm, variant)
+    wp, wn = _workspace(workspace, A_q.device, nbytes)
+    rc = lib().w8_grouped_gemm(fmt, _ptr(A_q), _ptr(A_scale), _ptr(W_q), _ptr(W_scale), _ptr(out),
+                               _ptr(expert_offsets), E, T, N, K, mm, variant, wp, wn, _stream(stream))
+    _check("w8_grouped_gemm", rc)
     return out
 
 

@@ -233,6 +233,33 @@ W8_API int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant);
 W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int N, int K, int variant,
                       void* workspace, size_t ws_bytes, w8_stream_t stream);
 
+/* Grouped (mixture-of-experts) scaled GEMM.  (The pages name mixture-of-experts models
+ * as the next target of the unified linear backend -- "Helion nel backend vLLM: un
+ * solo GEMM, tuning per forma e guadagni fino al 10%", last paragraph -- without a
+ * formula; this is the plain reading: the experts' GEMMs over tokens already routed.)
+ *   A_q [T, K] 8-bit codes, A_scale [T] fp32: the tokens (or token copies, one per
+ *       chosen expert) sorted by expert; rows [off[e], off[e+1]) belong to expert e;
+ *   expert_offsets int32 [E + 1] in device memory, rising from off[0] >= 0 to off[E]
+ *       <= T (read by the kernel after any programmatic-dependent-launch wait, so the
+ *       routing kernel ahead may write them); offsets that do not rise within [0, T]
+ *       compute nothing and record W8_ERR_INVALID_ARG in the device status word;
+ *   W_q [E, N, K] codes, W_scale [E, N] fp32 per expert and output channel;
+ *   out [T, N] bf16: row t = bf16(sum_k A[t,k] W_e[n,k] * A_scale[t] * W_scale[e,n]) for
+ *       the expert e owning row t (FP8-dynamic or W8A8-INT8, as w8_gemm); rows no expert
+ *       owns are not written.
+ * The kernel is the Swap-AB GEMM with the balanced partition: every CTA counts the
+ * experts' tiles from the offsets and deals out the units of the experts that have
+ * tokens, so empty experts cost nothing.  max_tokens_per_expert (<= T) bounds the tokens
+ * of one expert; it picks the token tile (AUTO) and sizes the workspace
+ * (w8_grouped_gemm_workspace_size; same rules as w8_gemm's).  An explicit variant must
+ * be Swap-AB with W8_V_STREAM. */
+W8_API int w8_grouped_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
+                           void* out, const int* expert_offsets, int E, int T, int N, int K,
+                           int max_tokens_per_expert, int variant, void* workspace, size_t ws_bytes,
+                           w8_stream_t stream);
+W8_API size_t w8_grouped_gemm_workspace_size(int fmt, int E, int T, int N, int K, int max_tokens_per_expert,
+                                             int variant);
+
 /* Query/key rms_norm + rotary embedding on the merged attention projection ("PyTorch
  * integra Helion en vLLM para acelerar inferencia FP8", section "Kernels Helion
  * implementados": fused_qk_norm_rope; named there without a formula).  Reading:
