@@ -283,6 +283,70 @@ def time_graph(fn, steps, warmup, world):
     return ms, launches
 
 
+def time_extras(dev, peak):
+    """Device time of the other hot-path kernels on their own (CUDA graph of a few launches
+    over inputs rotated past L2): the query/key rms_norm + rotary embedding at prefill size,
+    and the grouped (mixture-of-experts) GEMM at a decode routing.  HBM roofline fractions
+    against the same measured copy peak."""
+    import torch
+    from bit_quantized_gemm_token_b200 import w8
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+    res = {}
+    # qk norm + rope: 4096 tokens, 32 query / 8 key-value heads of 128 (in place)
+    T, Hq, Hkv, D = 4096, 32, 8, 128
+    bufs = [(torch.randn(T, (Hq + 2 * Hkv) * D, device=dev, generator=g)).to(torch.bfloat16) for _ in range(3)]
+    qw = (torch.rand(D, device=dev, generator=g) + 0.5).to(torch.bfloat16)
+    kw = (torch.rand(D, device=dev, generator=g) + 0.5).to(torch.bfloat16)
+    pos = torch.randint(0, 8192, (T,), device=dev, generator=g)
+    ang = torch.rand(8192, D // 2, device=dev, generator=g) * 6.283
+    table = torch.cat([ang.cos(), ang.sin()], dim=1).float()
+
+    def qk():
+        for b in bufs:
+            w8.w8_qk_norm_rope(b, Hq, Hkv, D, qw, kw, table, pos, out=b, stream=torch.cuda.current_stream())
+        return len(bufs)
+    ms, n = time_graph(qk, 5, 3, 1)
+    us = ms * 1e3 / n
+    byts = T * (Hq + Hkv) * D * 2 * 2 + T * D * 4
+    res["qk_norm_rope"] = {"shape": "T=%d Hq=%d Hkv=%d D=%d, in place" % (T, Hq, Hkv, D), "us": round(us, 2),
+                           "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+                           "frac": round(byts / (us * 1e-6) / 1e9 / peak, 4), "bytes": byts}
+    # grouped GEMM: 128 experts of 1536 x 2048 (FP8), 4 tokens routed to 8 experts each
+    E, N, K, M, top = 128, 1536, 2048, 4, 8
+    sets = []
+    for _ in range(2):
+        wb = (torch.randn(E * N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+        Wq, sW = w8.w8_quant_per_token(wb, w8.W8_Q_FP8)
+        sets.append((Wq.view(E, N, K), sW.view(E, N)))
+        del wb
+    choice = torch.stack([torch.randperm(E, device=dev, generator=g)[:top] for _ in range(M)]).flatten()
+    counts = torch.bincount(choice, minlength=E)
+    off = torch.zeros(E + 1, dtype=torch.int32, device=dev)
+    off[1:] = torch.cumsum(counts, 0).to(torch.int32)
+    rows = M * top
+    A = (torch.randn(rows, K, device=dev, generator=g)).to(torch.bfloat16)
+    Aq, sA = w8.w8_quant_per_token(A, w8.W8_Q_FP8)
+    out = torch.empty(rows, N, dtype=torch.bfloat16, device=dev)
+    ws = w8.Workspace(dev)
+    active = int((counts > 0).sum().item())
+
+    def grouped():
+        for Wq, sW in sets:
+            w8.w8_grouped_gemm(w8.W8_FMT_FP8_DYN, Aq, sA, Wq, sW, off, max_tokens_per_expert=M, out=out,
+                               variant=w8.W8_VARIANT_AUTO | w8.W8_V_PDL, workspace=ws)
+        return len(sets)
+    ms, n = time_graph(grouped, 5, 3, 1)
+    us = ms * 1e3 / n
+    byts = active * N * K + rows * K + 4 * active * N + 4 * rows + 2 * rows * N
+    res["grouped_gemm"] = {"shape": "E=%d N=%d K=%d, %d tokens x top-%d -> %d active experts" % (E, N, K, M, top, active),
+                           "us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+                           "frac": round(byts / (us * 1e-6) / 1e9 / peak, 4), "bytes": byts}
+    del sets
+    torch.cuda.empty_cache()
+    return res
+
+
 def time_e2e(wl, steps, warmup, world):
     """Same step through the public API with host buffers: every step copies all the
     step's activations from one pinned host buffer to the device (one copy), runs the
@@ -467,6 +531,8 @@ def run_ours(args):
         out["e2e"] = e2e
     if detail:
         out["detail"] = detail
+    if rank == 0 and not args.no_extras:
+        out["other_kernels"] = time_extras(dev, peak)
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(shapes, ms, target_s=args.cpu_seconds)
     if rank == 0:
@@ -518,6 +584,7 @@ def main():
     ap.add_argument("--single", default="", help="KxN: time one shape only (profiling case)")
     ap.add_argument("--m", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip timing the qk-norm/rope and grouped kernels")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
