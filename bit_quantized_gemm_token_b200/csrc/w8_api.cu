@@ -423,7 +423,9 @@ int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, c
     if (!qkv || !out || !q_weight || !k_weight || !cos_sin || !positions) return W8_ERR_INVALID_ARG;
     if (T < 0 || Hq < 0 || Hkv < 0 || max_pos <= 0 || !(eps >= 0.0f)) return W8_ERR_INVALID_ARG;
     if (D != 64 && D != 128 && D != 256) return W8_ERR_UNSUPPORTED;
-    if (!aligned(qkv, 2) || !aligned(out, 2) || !aligned(cos_sin, 4) || !aligned(positions, 8)) return W8_ERR_ALIGNMENT;
+    if (!aligned(qkv, 8) || !aligned(out, 8) || !aligned(q_weight, 8) || !aligned(k_weight, 8) || !aligned(cos_sin, 4) ||
+        !aligned(positions, 8))
+        return W8_ERR_ALIGNMENT;
     int rc = check_device(nullptr);
     if (rc != W8_OK) return rc;
     return launch_qk_norm_rope(qkv, out, T, Hq, Hkv, D, q_weight, k_weight, cos_sin, max_pos,

@@ -225,7 +225,8 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     maps.R = tR;
     maps.C = tC;
     cudaError_t e = cudaErrorInvalidValue;
-    if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, s);
+    if (p.grouped)                 e = launch_grouped(p, maps, args, s);
+    else if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, s);
     else if (p.bm == 64)           e = launch_bm64(p, maps, args, s);
     else if (p.fmt == W8_FMT_INT8) e = launch_i8(p, maps, args, s);
     else                           e = launch_f8(p, maps, args, s);
@@ -364,6 +365,7 @@ int gemm_occupancy(const GemmPlan& p, int* n)
     GemmArgs args = {};
     cudaError_t e = cudaErrorInvalidValue;
     if (p.fq)                      e = launch_fq(p, maps, args, nullptr);
+    else if (p.grouped)            e = launch_grouped(p, maps, args, nullptr);
     else if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, nullptr);
     else if (p.bm == 64)           e = launch_bm64(p, maps, args, nullptr);
     else if (p.fmt == W8_FMT_INT8) e = launch_i8(p, maps, args, nullptr);
@@ -376,7 +378,7 @@ int gemm_occupancy(const GemmPlan& p, int* n)
 int gemm_device_status(int clear)
 {
     int first = 0;
-    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq}) {
+    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq, status_grouped}) {
         const int v = f(clear);
         if (v == W8_ERR_CUDA) return v;
         if (v != 0 && first == 0) first = v;

@@ -301,7 +301,7 @@ __device__ __forceinline__ bool first_epi_thread(unsigned t) { return t == 64; }
 // "unit" of the partition is one stage block of KPS K blocks of one output tile.
 // Accumulator row r of a BM = 64 MMA lives in TMEM lane (r % 16) + 32 * (r / 16); of a
 // BM = 128 MMA in lane r.
-template <int BM, int BN, int KIND, bool BLOCK, int KPS, bool FQ = false>
+template <int BM, int BN, int KIND, bool BLOCK, int KPS, bool FQ = false, bool GRP = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC, const GemmArgs a)
 {
@@ -400,9 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ahead, hence after the wait), as prefix sums in shared memory; every CTA derives the
     // same balanced partition of the units of the experts that have tokens
     int* s_gtile = reinterpret_cast<int*>(tmem_slot + 4);     // [g_E + 1] tile prefix
-    int* s_goff = s_gtile + (a.grouped ? a.g_E + 1 : 0);       // [g_E + 1] clamped offsets
+    int* s_goff = s_gtile + (GRP ? a.g_E + 1 : 0);             // [g_E + 1] clamped offsets
     long long U = a.units;
-    if (a.grouped) {
+    if (GRP) {
         ptx::grid_dep_wait();
         if (warp == 0) {
             const int E = a.g_E, T = a.rows_C;
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // every CTA of the partition must own at least one unit (a split tile is finished by
     // its contributors, consecutive CTAs): with fewer units than CTAs the rest idle
-    const long long Gp = (a.grouped && U < a.G) ? U : a.G;
+    const long long Gp = (GRP && U < a.G) ? U : a.G;
     const long long u0 = ((long long)blockIdx.x < Gp) ? unit_begin(a, blockIdx.x, U, Gp) : U;
     const long long u1 = ((long long)blockIdx.x < Gp) ? unit_begin(a, blockIdx.x + 1, U, Gp) : U;
     // tile t -> weight tile rt, token tile ct, the rows they start at in W and A, and the
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // sit c_shift columns into it.
     auto tile_loc = [&](int t, int& rt, int& ct, int& r_off, int& c_off, int& c_valid, int& c_shift) {
         c_shift = 0;
-        if (!a.grouped) {
+        if (!GRP) {
             rt = t / a.c_tiles;
             ct = t % a.c_tiles;
             r_off = 0;
@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // this one, the producer requests the weight boxes of the first `pre` stages
             // (weights are never the output of work in flight; the epilogue warps prefetch
             // the next units' weights into L2); the activation boxes follow after the wait.
-            const int pre = (a.pdl && !a.grouped) ? (int)(n < S ? n : S) : 0;
+            const int pre = (a.pdl && !GRP) ? (int)(n < S ? n : S) : 0;
             for (int i = 0; i < pre; ++i) issue(i, u0 + i, a.swap != 0, a.swap == 0, true);
             ptx::grid_dep_wait();
             if (FQ) {
@@ -627,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
-        if (a.pdl && !FQ && !a.grouped) {
+        if (a.pdl && !FQ && !GRP) {
             // Idle until the first accumulator is ready: prefetch into L2 the weight rows
             // of the kL2Ahead units that follow the producer's first stages, so that the
             // weight stream keeps HBM busy while the kernels ahead of this one finish.
@@ -1192,10 +1192,10 @@ struct GemmMaps {
     int* occupancy = nullptr;   // when set: report resident CTAs per SM instead of launching
 };
 
-template <int BM, int BN, int KIND, bool BLOCK, int KPS, bool FQ = false>
+template <int BM, int BN, int KIND, bool BLOCK, int KPS, bool FQ = false, bool GRP = false>
 cudaError_t launch_one(const GemmPlan& p, const GemmMaps& maps, const GemmArgs& args, cudaStream_t s)
 {
-    auto kern = gemm_kernel<BM, BN, KIND, BLOCK, KPS, FQ>;
+    auto kern = gemm_kernel<BM, BN, KIND, BLOCK, KPS, FQ, GRP>;
     // the large dynamic shared-memory limit is a per-device function attribute
     static bool configured[64] = {};
     static std::mutex mu;
@@ -1255,11 +1255,13 @@ cudaError_t launch_i8(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, c
 cudaError_t launch_block(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_bm64(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_fq(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_grouped(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 int status_f8(int clear);
 int status_i8(int clear);
 int status_block(int clear);
 int status_bm64(int clear);
 int status_fq(int clear);
+int status_grouped(int clear);
 
 }  // namespace gemm
 }  // namespace w8

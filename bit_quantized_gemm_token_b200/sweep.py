@@ -52,7 +52,8 @@ def candidates(fmt, M, N, K, quick=False):
     if not block:
         # Standard form, 64-row token tile, weights in the MMA's N slot
         for bn in (128, 256):
-            parts = [("stream", 1), ("split", 1), ("split", 2), ("split", 4), ("split", 8), ("cluster", 2), ("cluster", 4)]
+            parts = [("stream", 1), ("split", 1), ("split", 2), ("split", 4), ("split", 8), ("cluster", 2), ("cluster", 4),
+                     ("cluster", 8)]
             for kind, arg in parts:
                 for kps in (1, 2):
                     for stages in ((0,) if quick else (0, 2, 3, 4)):

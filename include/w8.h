@@ -275,7 +275,8 @@ W8_API size_t w8_grouped_gemm_workspace_size(int fmt, int E, int T, int N, int K
  *   positions int64 [T] in [0, max_pos): a position outside records W8_ERR_INVALID_ARG
  *             in the device status word (w8_device_status) and leaves that token's
  *             query and key heads unwritten.
- * D must be 64, 128 or 256 (W8_ERR_UNSUPPORTED otherwise). */
+ * D must be 64, 128 or 256 (W8_ERR_UNSUPPORTED otherwise); qkv, out and the weights
+ * 8-byte aligned, cos_sin 4-byte, positions 8-byte (W8_ERR_ALIGNMENT otherwise). */
 W8_API int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
                            const void* k_weight, const float* cos_sin, int max_pos, const int64_t* positions,
                            float eps, w8_stream_t stream);
