@@ -57,6 +57,24 @@ def test_bad_arguments_rejected_before_device(L):
     assert L.w8_rmsnorm_quant(p16, NULL, ctypes.c_float(1e-6), 1, 16, 16, p16, p16, NULL) == w8.W8_ERR_INVALID_ARG
     assert L.w8_silu_mul_quant(p16, 1, 16, 16, p16, p16, NULL) == w8.W8_ERR_INVALID_ARG   # ld < 2I
     assert L.w8_gemm_i32_debug(p16, p16, NULL, 1, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    # quantize + GEMM: null input, row stride below K, misaligned x
+    assert L.w8_linear(0, NULL, 16, p16, p16, p16, 1, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    assert L.w8_linear(0, p16, 8, p16, p16, p16, 1, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_INVALID_ARG
+    assert L.w8_linear(0, podd, 16, p16, p16, p16, 1, 16, 16, 0, NULL, 0, NULL) == w8.W8_ERR_ALIGNMENT
+    assert L.w8_linear_debug(0, p16, 16, p16, p16, p16, 1, 16, 16, 0, NULL, 0, NULL, NULL, NULL) == \
+        w8.W8_ERR_INVALID_ARG
+    # grouped GEMM: no experts, no offsets, more tokens per expert than rows is clamped but E = 0 is not
+    assert L.w8_grouped_gemm(0, p16, p16, p16, p16, p16, p16, 0, 8, 16, 16, 8, 0, NULL, 0, NULL) == \
+        w8.W8_ERR_INVALID_ARG
+    assert L.w8_grouped_gemm(0, p16, p16, p16, p16, p16, NULL, 2, 8, 16, 16, 8, 0, NULL, 0, NULL) == \
+        w8.W8_ERR_INVALID_ARG
+    # query/key norm + rotary: head size 96 is not supported, misaligned qkv
+    assert L.w8_qk_norm_rope(p16, p16, 1, 2, 1, 96, p16, p16, p16, 8, p16, ctypes.c_float(1e-6), NULL) == \
+        w8.W8_ERR_UNSUPPORTED
+    assert L.w8_qk_norm_rope(ctypes.c_void_p((1 << 20) + 2), p16, 1, 2, 1, 128, p16, p16, p16, 8, p16,
+                             ctypes.c_float(1e-6), NULL) == w8.W8_ERR_ALIGNMENT
+    assert L.w8_qk_norm_rope(NULL, p16, 1, 2, 1, 128, p16, p16, p16, 8, p16, ctypes.c_float(1e-6), NULL) == \
+        w8.W8_ERR_INVALID_ARG
 
 
 def test_valid_call_without_device_reports_no_device(L):
@@ -66,6 +84,23 @@ def test_valid_call_without_device_reports_no_device(L):
     p16 = ctypes.c_void_p(1 << 20)
     assert L.w8_quant_per_token(0, p16, 1, 16, 16, p16, p16, 0, 0, NULL) == w8.W8_ERR_NO_DEVICE
     assert L.w8_gemm(0, p16, p16, p16, p16, p16, 1, 128, 128, 0, NULL, 0, NULL) == w8.W8_ERR_NO_DEVICE
+
+
+def test_linear_and_grouped_planning(L):
+    w8.w8_clear_table()
+    # w8_linear runs the quantizer and the GEMM unless the one-kernel form is asked for
+    v = w8.w8_linear_resolve(0, 4, 4096, 4096)
+    assert not (v & w8.W8_V_FUSED)
+    vf = w8.w8_linear_resolve(0, 4, 4096, 4096, w8.variant(True, 4, 16, cluster=True) | w8.W8_V_FUSED)
+    assert vf & w8.W8_V_FUSED
+    assert L.w8_linear_resolve(0, 100, 4096, 4096, w8.variant(False, 1, 128) | w8.W8_V_FUSED) == w8.W8_ERR_UNSUPPORTED
+    # the two-kernel workspace keeps the codes past the 256 KiB counter area
+    assert w8.w8_linear_workspace_size(0, 4, 4096, 4096, w8.variant(True, 1, 16)) >= 65536 * 4 + 4 * 4096
+    # grouped GEMM: counter area + one partial slot pair per CTA; Standard tiles are refused
+    n = w8.w8_grouped_gemm_workspace_size(0, 64, 32, 1536, 2048, 4)
+    assert n >= 65536 * 4 + 148 * 2 * 16 * 128 * 4
+    assert L.w8_grouped_gemm_workspace_size(0, 64, 32, 1536, 2048, 4, w8.variant(False, 1, 128, stream=True)) == \
+        ctypes.c_size_t(-1).value
 
 
 def test_variant_resolution_and_workspace(L):
