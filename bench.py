@@ -344,7 +344,39 @@ def time_extras(dev, peak):
                            "frac": round(byts / (us * 1e-6) / 1e9 / peak, 4), "bytes": byts}
     del sets
     torch.cuda.empty_cache()
+    # prefill GEMM (tensor-bound): FP8-dynamic, M = 4096 tokens on the gate_up shape
+    M, K, N = 4096, 4096, 24576
+    Aq, sA = w8.w8_quant_per_token(torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16), w8.W8_Q_FP8)
+    Wq, sW = w8.w8_quant_per_token((torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16), w8.W8_Q_FP8)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    flop = 2.0 * M * N * K
+    fp8_peak = 2.0 * peak_tflops()          # dense fp8 = 2 x the measured dense bf16 figure
+    best = None
+    for name, v in [("auto", w8.W8_VARIANT_AUTO), ("standard 128x256", w8.variant(False, 1, 256)),
+                    ("standard 128x128", w8.variant(False, 1, 128)), ("balanced 128x256", w8.variant(False, 1, 256, stream=True))]:
+        def pre():
+            for _ in range(3):
+                w8.w8_gemm(w8.W8_FMT_FP8_DYN, Aq, sA, Wq, sW, out=out, variant=v | w8.W8_V_PDL, workspace=ws)
+            return 3
+        ms, n = time_graph(pre, 3, 2, 1)
+        tf = flop / (ms * 1e-3 / n) / 1e12
+        if best is None or tf > best[1]:
+            best = (name, tf, ms * 1e3 / n)
+    res["prefill_gemm"] = {"shape": "FP8-dynamic M=%d K=%d N=%d" % (M, K, N), "variant": best[0], "us": round(best[2], 1),
+                           "TFLOP/s": round(best[1], 1), "peak_TFLOP/s": round(fp8_peak, 1),
+                           "frac": round(best[1] / fp8_peak, 4),
+                           "peak_source": "2 x measured dense bf16 (burst)"}
+    del Aq, Wq, out
+    torch.cuda.empty_cache()
     return res
+
+
+def peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return float(json.load(fh)["bf16_tflops"])
+    return 1590.0
 
 
 def time_e2e(wl, steps, warmup, world):
