@@ -63,9 +63,9 @@ int table_lookup(int fmt, int N, int K, int M)
 
 namespace {
 
-// Built-in rule when the table has no entry: Swap-AB with the narrowest token tile for
-// decode-sized M, the Standard 128 x 128 tile otherwise; always the balanced partition
-// (weights are streamed evenly by every SM; the partial-sum traffic stays in L2).
+// Built-in rule when the table has no entry: Swap-AB with the narrowest token tile and the
+// balanced partition for decode-sized M (weights streamed evenly by every SM; the
+// partial-sum traffic stays in L2); the Standard form with whole tiles for prefill.
 // Grouped GEMM default: Swap-AB over the balanced partition with the narrowest token tile
 // that holds an expert's largest token count (64 beyond that: several token tiles).
 int grouped_variant(int max_m)
@@ -80,7 +80,10 @@ int builtin_variant(int fmt, int M)
     if (M <= 16) return W8_VARIANT(1, 0, kTileBN16, 1);
     if (M <= 32) return W8_VARIANT(1, 0, kTileBN32, 1);
     if (M <= 64) return W8_VARIANT(1, 0, kTileBN64, 1);
-    return W8_VARIANT(0, 0, block ? kTileBN64 : kTileBN128, 1);
+    // prefill: tensor-bound; every MMA costs about the same issue time whatever its N, so
+    // the widest weight tile (256; 64 for Block-FP8, whose promotion keeps the tile in
+    // registers) over whole-tile loops
+    return block ? W8_VARIANT(0, 0, kTileBN64, 1) : W8_VARIANT(0, 0, kTileBN256, 0);
 }
 
 int resolve(int fmt, int M, int N, int K, int variant, int sms, GemmPlan* plan)
