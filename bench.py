@@ -368,9 +368,130 @@ def time_extras(dev, peak):
                            "TFLOP/s": round(best[1], 1), "peak_TFLOP/s": round(fp8_peak, 1),
                            "frac": round(best[1] / fp8_peak, 4),
                            "peak_source": "2 x measured dense bf16 (burst)", "variants_TFLOP/s": tried}
+    # the same shape in W8A8-INT8 (int8 tensor cores, int32 accumulation), built-in variant
+    xa = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+    xw = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+    Aq, sA = w8.w8_quant_per_token(xa, w8.W8_Q_INT8)
+    Wq, sW = w8.w8_quant_per_token(xw, w8.W8_Q_INT8)
+    del xa, xw
+
+    def pre_i8():
+        for _ in range(3):
+            w8.w8_gemm(w8.W8_FMT_INT8, Aq, sA, Wq, sW, out=out, variant=w8.W8_VARIANT_AUTO | w8.W8_V_PDL, workspace=ws)
+        return 3
+    ms, n = time_graph(pre_i8, 3, 2, 1)
+    tf = flop / (ms * 1e-3 / n) / 1e12
+    res["prefill_gemm_int8"] = {"shape": "W8A8-INT8 M=%d K=%d N=%d" % (M, K, N), "us": round(ms * 1e3 / n, 1),
+                                "TOP/s": round(tf, 1), "peak_TOP/s": round(fp8_peak, 1), "frac": round(tf / fp8_peak, 4),
+                                "peak_source": "2 x measured dense bf16 (burst)"}
     del Aq, Wq, out
     torch.cuda.empty_cache()
+    # the other formats' decode chains (quantizer + GEMM per layer), like the step above
+    res["int8_decode"] = format_chain(dev, g, w8, w8.W8_FMT_INT8, SHAPES, [1, 8, 32], peak)
+    res["block_fp8_decode"] = format_chain(dev, g, w8, w8.W8_FMT_BLOCK_FP8,
+                                           [(5120, 10240), (5120, 51200), (25600, 5120), (4096, 6144)], [1, 8, 32], peak)
+    res["mlp_chain"] = mlp_chain(dev, g, w8, peak, fp8_peak)
     return res
+
+
+def mlp_chain(dev, g, w8, peak, fp8_peak):
+    """The MLP block hidden 4096 / intermediate 12288 in FP8-dynamic: rms_norm + quant,
+    gate_up GEMM, silu_and_mul + quant, down GEMM (AUTO + PDL, one CUDA graph per token
+    count, two weight copies in rotation).  Decode token counts in TB/s of algorithmic
+    bytes, prefill ones in TFLOP/s of the two GEMMs."""
+    import torch
+    H, I = 4096, 12288
+    gamma = (torch.rand(H, device=dev, generator=g) + 0.5).to(torch.bfloat16)
+    Wgu, Wd = [], []
+    for _ in range(2):
+        Wgu.append(w8.w8_quant_per_token((torch.randn(2 * I, H, device=dev, generator=g) * 0.02).to(torch.bfloat16)))
+        Wd.append(w8.w8_quant_per_token((torch.randn(H, I, device=dev, generator=g) * 0.02).to(torch.bfloat16)))
+    ws = w8.Workspace(dev)
+    v = w8.W8_VARIANT_AUTO | w8.W8_V_PDL
+    out = {}
+    for M in (1, 8, 32, 256, 1024, 4096):
+        x = torch.randn(M, H, device=dev, generator=g).to(torch.bfloat16)
+        q1 = torch.empty(M, H, dtype=torch.float8_e4m3fn, device=dev)
+        s1 = torch.empty(M, device=dev)
+        gu = torch.empty(M, 2 * I, dtype=torch.bfloat16, device=dev)
+        q2 = torch.empty(M, I, dtype=torch.float8_e4m3fn, device=dev)
+        s2 = torch.empty(M, device=dev)
+        y = torch.empty(M, H, dtype=torch.bfloat16, device=dev)
+        reps = 4 if M <= 32 else 2
+
+        def chain():
+            for r in range(reps):
+                w8.w8_rmsnorm_quant(x, gamma, 1e-6, q=q1, scale=s1)
+                w8.w8_gemm(0, q1, s1, Wgu[r % 2][0], Wgu[r % 2][1], out=gu, variant=v, workspace=ws)
+                w8.w8_silu_mul_quant(gu, q=q2, scale=s2)
+                w8.w8_gemm(0, q2, s2, Wd[r % 2][0], Wd[r % 2][1], out=y, variant=v, workspace=ws)
+            return 4 * reps
+        ms, _ = time_graph(chain, 5, 3, 1)
+        us = ms * 1e3 / reps
+        if M <= 32:
+            byts = (2 * M * H + 2 * H + M * H + 4 * M) + gemm_bytes(M, 2 * I, H) \
+                + (2 * M * 2 * I + M * I + 4 * M) + gemm_bytes(M, H, I)
+            gbs = byts / (us * 1e-6) / 1e9
+            out["M=%d" % M] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        else:
+            tf = 2.0 * M * (H * 2 * I + I * H) / (us * 1e-6) / 1e12
+            out["M=%d" % M] = {"us": round(us, 1), "TFLOP/s": round(tf, 1), "frac": round(tf / fp8_peak, 4)}
+        del x, q1, s1, gu, q2, s2, y
+    del Wgu, Wd
+    torch.cuda.empty_cache()
+    out["shape"] = "hidden 4096, intermediate 12288, FP8-dynamic; decode frac of the copy peak, prefill of 2 x dense bf16"
+    return out
+
+
+def format_chain(dev, g, w8, fmt, shapes, ms, peak):
+    """TB/s of a graph of (activation quantizer, GEMM) pairs over the shapes and token
+    counts in format fmt (W8A8-INT8 per token, or Block-FP8 with 1 x 128 activation
+    groups and 128 x 128 weight blocks), two weight copies per shape in rotation."""
+    import torch
+    block = fmt >= w8.W8_FMT_BLOCK_FP8
+    W = {}
+    for (K, N) in shapes:
+        for c in range(2):
+            wb = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+            W[(K, N, c)] = w8.w8_quant_weight_block(wb) if block else w8.w8_quant_per_token(wb, w8.W8_Q_INT8)
+            del wb
+    X = {(M, K): (torch.randn(M, K, device=dev, generator=g)).to(torch.bfloat16) for M in ms for (K, N) in shapes}
+    A = {}
+    for (M, K), x in X.items():
+        A[(M, K)] = (w8.w8_quant_per_token(x, w8.W8_Q_FP8, group=128) if block else w8.w8_quant_per_token(x, w8.W8_Q_INT8))
+    O = {(M, N): torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in ms for (K, N) in shapes}
+    ws = w8.Workspace(dev)
+    v = w8.W8_VARIANT_AUTO | w8.W8_V_PDL
+    byts = 0
+    for M in ms:
+        for (K, N) in shapes:
+            if block:   # 128 x 128 weight-block scales, 1 x 128 activation-group scales
+                kb = K // 128
+                byts += (N * K + 4 * ((N + 127) // 128) * kb + M * K + 4 * M * kb + 2 * M * N
+                         + 2 * M * K + M * K + 4 * M * kb)
+            else:
+                byts += gemm_bytes(M, N, K) + quant_bytes(M, K)
+
+    def chain():
+        n = 0
+        for mi, M in enumerate(ms):
+            for si, (K, N) in enumerate(shapes):
+                q, sc = A[(M, K)]
+                if block:
+                    w8.w8_quant_per_token(X[(M, K)], w8.W8_Q_FP8, group=128, q=q, scale=sc)
+                else:
+                    w8.w8_quant_per_token(X[(M, K)], w8.W8_Q_INT8, q=q, scale=sc)
+                Wq, sW = W[(K, N, (mi + si) % 2)]
+                w8.w8_gemm(fmt, q, sc, Wq, sW, out=O[(M, N)], variant=v, workspace=ws)
+                n += 2
+        return n
+    ms_step, _ = time_graph(chain, 5, 3, 1)
+    tbs = byts / (ms_step * 1e-3) / 1e12
+    out = {"shapes_KxN": ["%dx%d" % s for s in shapes], "M": ms, "us_per_step": round(ms_step * 1e3, 1),
+           "TB/s": round(tbs, 3), "frac": round(tbs * 1e3 / peak, 4)}
+    del W, X, A, O
+    torch.cuda.empty_cache()
+    return out
 
 
 def peak_tflops():
