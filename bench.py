@@ -677,7 +677,8 @@ def run_ours(args):
     peak, peak_kind = load_peaks()
     achieved = gb / (ms_gemm * 1e-3) / 1e9    # GB/s, GEMM kernels alone
     n_gemm_per_step = len(shapes) * len(ms)
-    traffic = traffic_from_profile()
+    # the committed capture is of the decode sweep's GEMM launches: no figure for other workloads
+    traffic = traffic_from_profile() if (not args.single and args.path == "pair") else None
     value = job_throughput(world, gb + qb, ms_step)
     out = {
         "metric": METRIC, "value": round(value, 4), "unit": "TB/s", "n_gpus": world, "steps": args.steps,
