@@ -1,6 +1,7 @@
 // w8_gemm.cu -- host side of the scaled 8-bit GEMM: tensor maps, planning of the
 // variant (tiles, partition, pipeline depth, workspace) and dispatch to the kernel
-// families (w8_gemm_f8.cu, w8_gemm_i8.cu, w8_gemm_block.cu, w8_gemm_bm64.cu).  The
+// families (w8_gemm_f8.cu, w8_gemm_i8.cu, w8_gemm_block.cu, w8_gemm_bm64.cu,
+// w8_gemm_fq.cu, w8_gemm_grouped.cu, and the CTA-pair loop of w8_gemm_pair.cu).  The
 // kernel itself and what it computes are described in w8_gemm_kernel.cuh.
 #include "w8_gemm_kernel.cuh"
 
@@ -104,6 +105,38 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
     q.bm = (variant & W8_V_BM64) ? 64 : 128;
     q.pfix = (variant & W8_V_PFIX) ? 1 : 0;
     if (lg > 8) return W8_ERR_UNSUPPORTED;
+    if (variant & W8_V_PAIR) {
+        // 256 x 256 tiles on CTA pairs: Standard full-K loop, FP8-dynamic / INT8
+        if (block || q.swap || q.stream || lg != 0 || q.cluster || q.bm != 128 || q.pfix || tid != kTileBN256 ||
+            kps > 1)
+            return W8_ERR_UNSUPPORTED;
+        if (stages == 0) stages = 6;
+        if (stages < 2) return W8_ERR_UNSUPPORTED;
+        q.pair = 1;
+        q.bn = 256;
+        q.split = 1;
+        q.kps = 1;
+        q.stages = stages;
+        q.kbs = (K + 127) / 128;
+        q.nsb = q.kbs;
+        q.smem_bytes = 1024 + (size_t)stages * 2 * 128 * 128 + (size_t)(2 * stages + 5) * 8 + 16;
+        if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
+        q.rows_R = M;
+        q.rows_C = N;
+        q.r_tiles = (M + 255) / 256;
+        q.c_tiles = (N + 255) / 256;
+        q.tiles = q.r_tiles * q.c_tiles;
+        q.units = (long long)q.tiles * q.nsb;
+        const long long pairs_max = (sm_count > 0 ? sm_count : 148) / 2;
+        const long long pairs = q.tiles < pairs_max ? q.tiles : pairs_max;
+        if (pairs < 1) return W8_ERR_UNSUPPORTED;
+        q.G = (int)(2 * pairs);
+        q.align_tiles = 1;
+        q.ws_counters = 0;
+        q.ws_bytes = 0;
+        *p = q;
+        return W8_OK;
+    }
     // the 64-row tile holds tokens: Standard form, FP8 / INT8, weight tiles of 128 or 256 rows
     if (q.bm == 64 && (q.swap || block || (tid != kTileBN128 && tid != kTileBN256))) return W8_ERR_UNSUPPORTED;
     // cluster split: 2, 4 or 8 K chunks, one cluster (portable size) per tile
@@ -192,7 +225,8 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     const void* C = p.swap ? A_q : W_q;
     // the grouped form's weights are the experts' [N, K] matrices one after another
     if (!make_tmap(&tR, R, p.grouped ? p.rows_R * p.g_E : p.rows_R, p.K, p.bm)) return W8_ERR_CUDA;
-    if (!make_tmap(&tC, C, p.rows_C, p.K, p.bn)) return W8_ERR_CUDA;
+    // a CTA of a pair loads half of the 256 weight rows of a tile
+    if (!make_tmap(&tC, C, p.rows_C, p.K, p.pair ? 128 : p.bn)) return W8_ERR_CUDA;
 
     GemmArgs args = {};
     args.M = p.M; args.N = p.N; args.K = p.K;
@@ -226,6 +260,7 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     maps.C = tC;
     cudaError_t e = cudaErrorInvalidValue;
     if (p.grouped)                 e = launch_grouped(p, maps, args, s);
+    else if (p.pair)               e = launch_pair(p, maps, args, s);
     else if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, s);
     else if (p.bm == 64)           e = launch_bm64(p, maps, args, s);
     else if (p.fmt == W8_FMT_INT8) e = launch_i8(p, maps, args, s);
@@ -366,6 +401,7 @@ int gemm_occupancy(const GemmPlan& p, int* n)
     cudaError_t e = cudaErrorInvalidValue;
     if (p.fq)                      e = launch_fq(p, maps, args, nullptr);
     else if (p.grouped)            e = launch_grouped(p, maps, args, nullptr);
+    else if (p.pair)               e = launch_pair(p, maps, args, nullptr);
     else if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, nullptr);
     else if (p.bm == 64)           e = launch_bm64(p, maps, args, nullptr);
     else if (p.fmt == W8_FMT_INT8) e = launch_i8(p, maps, args, nullptr);
@@ -378,7 +414,7 @@ int gemm_occupancy(const GemmPlan& p, int* n)
 int gemm_device_status(int clear)
 {
     int first = 0;
-    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq, status_grouped}) {
+    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq, status_grouped, status_pair}) {
         const int v = f(clear);
         if (v == W8_ERR_CUDA) return v;
         if (v != 0 && first == 0) first = v;

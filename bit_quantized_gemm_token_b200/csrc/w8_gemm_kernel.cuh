@@ -1256,12 +1256,14 @@ cudaError_t launch_block(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a
 cudaError_t launch_bm64(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_fq(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_grouped(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_pair(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 int status_f8(int clear);
 int status_i8(int clear);
 int status_block(int clear);
 int status_bm64(int clear);
 int status_fq(int clear);
 int status_grouped(int clear);
+int status_pair(int clear);
 
 }  // namespace gemm
 }  // namespace w8

@@ -50,6 +50,7 @@ struct GemmPlan {
     int fq_full_rows; // fq: whole rows staged (per-token maxima without a cluster split)
     int grouped;      // mixture-of-experts form: M = all tokens, N per expert
     int g_E;          // grouped: experts
+    int pair;         // 256 x 256 tiles on CTA pairs (cta_group::2 MMA), Standard form
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile

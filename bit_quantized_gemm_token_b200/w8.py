@@ -41,13 +41,15 @@ W8_V_CLUSTER = 1 << 17
 W8_V_BM64 = 1 << 18
 W8_V_PFIX = 1 << 19
 W8_V_FUSED = 1 << 24
+W8_V_PAIR = 1 << 25
 W8_V_KPS_SHIFT = 20
 W8_V_CPS_SHIFT = 22
 TILE_BN = {16: 0, 32: 1, 64: 2, 128: 3, 256: 4}
 
 
 def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stages: int = 0, pdl: bool = False,
-            kps: int = 0, cps: int = 0, cluster: bool = False, bm64: bool = False, pfix: bool = False) -> int:
+            kps: int = 0, cps: int = 0, cluster: bool = False, bm64: bool = False, pfix: bool = False,
+            pair: bool = False) -> int:
     """Explicit variant word (the W8_VARIANT macro plus stages, PDL, K blocks per stage
     and CTAs per SM)."""
     lg = int(split).bit_length() - 1
@@ -67,6 +69,8 @@ def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stag
         v |= W8_V_BM64
     if pfix:
         v |= W8_V_PFIX
+    if pair:
+        v |= W8_V_PAIR
     return v
 
 
@@ -76,7 +80,8 @@ def describe(v: int) -> dict:
             "split_k": 1 << ((v >> W8_V_SPLIT_SHIFT) & 0xF), "bn": inv.get((v >> W8_V_TILE_SHIFT) & 0xF),
             "stages": (v >> W8_V_STAGES_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL),
             "kps": (v >> W8_V_KPS_SHIFT) & 0x3, "cps": (v >> W8_V_CPS_SHIFT) & 0x3,
-            "cluster": bool(v & W8_V_CLUSTER), "bm64": bool(v & W8_V_BM64), "pfix": bool(v & W8_V_PFIX)}
+            "cluster": bool(v & W8_V_CLUSTER), "bm64": bool(v & W8_V_BM64), "pfix": bool(v & W8_V_PFIX),
+            "pair": bool(v & W8_V_PAIR)}
 
 
 class W8Error(RuntimeError):

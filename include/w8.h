@@ -113,6 +113,14 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 block, so split_k must not exceed ceil(K / (128 * kps)).
  *   ctas/SM       bits 22..23, CTAs per SM for W8_V_STREAM and the Standard loop
  *                 (0 = 1).
+ *   W8_V_PAIR     Standard full-K tile loop (tile 256, split = 0, no W8_V_STREAM /
+ *                 W8_V_CLUSTER / W8_V_BM64; FP8-dynamic or INT8) over 256-token x
+ *                 256-weight-row tiles, each computed by a cluster of two CTAs on two SMs
+ *                 with one 256-row tensor-core MMA (cta_group::2).  Each CTA loads 128
+ *                 token rows and 128 weight rows per K block, and its tensor memory holds
+ *                 its 128 output rows; the pairs take whole tiles in contiguous runs.
+ *                 Stages default to 6.  Bit-identical to the one-CTA Standard loop (same
+ *                 products, same K order, one accumulator).  For prefill sizes.
  *   W8_V_PDL      launch with programmatic dependent launch: the kernel may start while
  *                 earlier kernels on the stream still run, and it reads weight tiles
  *                 (into shared memory and L2) before waiting for them.  Only legal when
@@ -132,6 +140,7 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 #define W8_V_BM64 (1 << 18)
 #define W8_V_PFIX (1 << 19)
 #define W8_V_FUSED (1 << 24)
+#define W8_V_PAIR (1 << 25)
 #define W8_V_KPS_SHIFT 20
 #define W8_V_CPS_SHIFT 22
 #define W8_VARIANT(swap, log2_split, tile, stream)                                            \

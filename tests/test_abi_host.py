@@ -111,12 +111,26 @@ def test_variant_resolution_and_workspace(L):
     assert d["swap_ab"] and d["stream"] and d["bn"] == 16
     assert w8.describe(w8.w8_gemm_resolve_variant(0, 32, 4096, 4096))["bn"] == 32
     assert not w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["swap_ab"]
+    # prefill past one 128-row token tile: CTA pairs (FP8 / INT8); Block-FP8 keeps its tile
+    assert w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["pair"]
+    assert w8.describe(w8.w8_gemm_resolve_variant(1, 256, 4096, 4096))["pair"]
+    assert not w8.describe(w8.w8_gemm_resolve_variant(0, 128, 4096, 4096))["pair"]
+    assert not w8.describe(w8.w8_gemm_resolve_variant(2, 4096, 4096, 4096))["pair"]
     # explicit variants are validated
     assert L.w8_gemm_resolve_variant(0, 8, 256, 1024, w8.variant(True, split=4, bn=16)) > 0
     assert L.w8_gemm_resolve_variant(0, 8, 256, 256, w8.variant(True, split=4, bn=16)) == w8.W8_ERR_UNSUPPORTED  # 4 > 2 K blocks
     assert L.w8_gemm_resolve_variant(2, 8, 256, 256, w8.variant(True, bn=128)) == w8.W8_ERR_UNSUPPORTED  # block needs BN <= 64
     assert L.w8_gemm_resolve_variant(0, 8, 256, 200, 0) == w8.W8_ERR_ALIGNMENT          # K % 16
     assert L.w8_gemm_resolve_variant(2, 8, 256, 144, 0) == w8.W8_ERR_ALIGNMENT          # block K % 128
+    # CTA pairs: Standard whole-tile loop with the 256 tile, FP8-dynamic / INT8 only
+    pair = w8.variant(False, 1, 256, pair=True)
+    for fmt in (0, 1):
+        assert L.w8_gemm_resolve_variant(fmt, 4096, 4096, 4096, pair) > 0
+        assert L.w8_gemm_workspace_size(fmt, 4096, 4096, 4096, pair) == 0
+    for fmt, v in ((2, pair), (0, w8.variant(True, 1, 256, pair=True)), (0, w8.variant(False, 2, 256, pair=True)),
+                   (0, w8.variant(False, 1, 128, pair=True)), (0, w8.variant(False, 1, 256, stream=True, pair=True)),
+                   (0, w8.variant(False, 1, 256, bm64=True, pair=True))):
+        assert L.w8_gemm_resolve_variant(fmt, 4096, 4096, 4096, v) == w8.W8_ERR_UNSUPPORTED
     # parallel fixup: 64-row token tile only, no cluster, at most one CTA per SM
     assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True)) > 0
     assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(True, 1, 16, stream=True, pfix=True)) == \

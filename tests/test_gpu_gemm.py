@@ -39,6 +39,8 @@ VARIANTS = {
     "bm64_256_stream_pfix_pdl": w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True, pdl=True, kps=1, stages=5),
     "bm64_128_split4_pfix_kps2": w8.variant(False, 4, 128, bm64=True, pfix=True, kps=2, stages=3),
     "bm64_256_split2_pfix": w8.variant(False, 2, 256, bm64=True, pfix=True, kps=1),
+    "pair256": w8.variant(False, 1, 256, pair=True),
+    "pair256_st3_pdl": w8.variant(False, 1, 256, pair=True, stages=3, pdl=True),
 }
 
 BLOCK_OK = {"auto", "swap16", "swap32_split2", "swap16_stream", "swap64_split4", "std64_split4", "std32_split8",
@@ -123,6 +125,22 @@ def test_split_k_up_to_256(orc):
             got = w8.w8_gemm_i32_debug(dev_codes(Aq, 1), dev_codes(Wq, 1), variant=v)
             torch.cuda.synchronize()
             assert np.array_equal(got.cpu().numpy().astype(np.int64), acc), (S, swap)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(1000, 5000, 384), (300, 40000, 256), (4096, 2048, 272), (257, 257, 128)])
+def test_pair_tiles(orc, fmt, M, N, K):
+    """256 x 256 tiles on CTA pairs at sizes with more tiles than pairs, ragged token and
+    weight tiles and a ragged K block: the oracle's outputs within the GEMM bound and,
+    for INT8, its int32 accumulators exactly."""
+    Aq, sA, Wq, sW, ref, acc = operands(orc, fmt, M, N, K)
+    for v in (w8.variant(False, 1, 256, pair=True), w8.variant(False, 1, 256, pair=True, pdl=True, stages=4)):
+        assert_bf16_close(run(fmt, Aq, sA, Wq, sW, v, M, N), ref, "pair %s" % ((M, N, K),))
+        if fmt == 1:
+            a32 = w8.w8_gemm_i32_debug(dev_codes(Aq, 1), dev_codes(Wq, 1), variant=v)
+            torch.cuda.synchronize()
+            assert np.array_equal(a32.cpu().numpy().astype(np.int64), acc)
+    assert w8.w8_device_status(clear=True) == 0
 
 
 def test_repeated_calls_reuse_workspace(orc):
