@@ -7,7 +7,7 @@
 // of two CTAs on two SMs with one tcgen05 MMA of M = 256 (cta_group::2):
 //   * each CTA loads, per 128-column K block, its own 128 token rows and 128 of the
 //     tile's 256 weight rows (32 KB per stage instead of the 48 KB a one-CTA 128 x 256
-//     tile needs), so the same shared memory holds six stages instead of four;
+//     tile needs), so the same shared memory holds five or six stages instead of four;
 //   * both CTAs' loads signal the leader's (rank 0) full barrier, on which the leader
 //     alone expects the bytes of both;
 //   * the leader issues the MMAs; they read the A rows and the B rows of both CTAs at the

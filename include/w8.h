@@ -119,8 +119,10 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 with one 256-row tensor-core MMA (cta_group::2).  Each CTA loads 128
  *                 token rows and 128 weight rows per K block, and its tensor memory holds
  *                 its 128 output rows; the pairs take whole tiles in contiguous runs.
- *                 Stages default to 6.  Bit-identical to the one-CTA Standard loop (same
- *                 products, same K order, one accumulator).  For prefill sizes.
+ *                 Stages default to 5.  The same sum as the one-CTA Standard loop: one
+ *                 accumulator over the whole K range, K blocks in order (INT8
+ *                 accumulators are exact).  For prefill sizes; with PDL the kernel waits
+ *                 for the kernels ahead before its first load.
  *   W8_V_PDL      launch with programmatic dependent launch: the kernel may start while
  *                 earlier kernels on the stream still run, and it reads weight tiles
  *                 (into shared memory and L2) before waiting for them.  Only legal when
