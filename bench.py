@@ -356,7 +356,7 @@ def time_extras(dev, peak):
     for name, v in [("auto", w8.W8_VARIANT_AUTO), ("standard 128x256", w8.variant(False, 1, 256)),
                     ("standard 128x128", w8.variant(False, 1, 128)), ("balanced 128x256", w8.variant(False, 1, 256, stream=True)),
                     ("CTA pairs 256x256", w8.variant(False, 1, 256, pair=True)),
-                    ("CTA pairs 256x256, 5 stages", w8.variant(False, 1, 256, pair=True, stages=5))]:
+                    ("CTA pairs 256x256, 6 stages", w8.variant(False, 1, 256, pair=True, stages=6))]:
         def pre():
             for _ in range(3):
                 w8.w8_gemm(w8.W8_FMT_FP8_DYN, Aq, sA, Wq, sW, out=out, variant=v | w8.W8_V_PDL, workspace=ws)
