@@ -82,12 +82,12 @@ int builtin_variant(int fmt, int M)
     if (M <= 64) return W8_VARIANT(1, 0, kTileBN64, 1);
     // prefill: tensor-bound; every MMA costs about the same issue time whatever its N, so
     // the widest weight tile (256; 64 for Block-FP8, whose promotion keeps the tile in
-    // registers) over whole-tile loops.  Past one 128-row token tile, 256 x 256 tiles on
-    // CTA pairs: a third less shared-memory traffic per MMA, hence deeper pipelines
-    // (1.71 -> 2.36 PFLOP/s on B200 at M = 4096, K = 4096, N = 24576, FP8)
+    // registers) over whole-tile loops.  FP8 / INT8: 256 x 256 tiles on CTA pairs, a
+    // third less shared-memory traffic per MMA, hence deeper pipelines (1.71 -> 2.36
+    // PFLOP/s on B200 at M = 4096, K = 4096, N = 24576); measured ahead of the one-CTA
+    // loops and of Swap-AB from M = 72 on (2x over the four dense shapes at M = 96)
     if (block) return W8_VARIANT(0, 0, kTileBN64, 1);
-    if (M > 128) return W8_VARIANT(0, 0, kTileBN256, 0) | W8_V_PAIR;
-    return W8_VARIANT(0, 0, kTileBN256, 0);
+    return W8_VARIANT(0, 0, kTileBN256, 0) | W8_V_PAIR;
 }
 
 int resolve(int fmt, int M, int N, int K, int variant, int sms, GemmPlan* plan)

@@ -111,10 +111,11 @@ def test_variant_resolution_and_workspace(L):
     assert d["swap_ab"] and d["stream"] and d["bn"] == 16
     assert w8.describe(w8.w8_gemm_resolve_variant(0, 32, 4096, 4096))["bn"] == 32
     assert not w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["swap_ab"]
-    # prefill past one 128-row token tile: CTA pairs (FP8 / INT8); Block-FP8 keeps its tile
+    # past 64 tokens: CTA pairs (FP8 / INT8); Block-FP8 keeps its tile
     assert w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["pair"]
     assert w8.describe(w8.w8_gemm_resolve_variant(1, 256, 4096, 4096))["pair"]
-    assert not w8.describe(w8.w8_gemm_resolve_variant(0, 128, 4096, 4096))["pair"]
+    assert w8.describe(w8.w8_gemm_resolve_variant(0, 65, 4096, 4096))["pair"]
+    assert not w8.describe(w8.w8_gemm_resolve_variant(0, 64, 4096, 4096))["pair"]
     assert not w8.describe(w8.w8_gemm_resolve_variant(2, 4096, 4096, 4096))["pair"]
     # explicit variants are validated
     assert L.w8_gemm_resolve_variant(0, 8, 256, 1024, w8.variant(True, split=4, bn=16)) > 0
