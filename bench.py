@@ -83,8 +83,9 @@ def traffic_from_profile():
     return d.get("dram_bytes_per_launch")
 
 
-class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+class SmiSampler:
+    """nvidia-smi clock / throttle sampling (100 ms) over the whole measurement: the
+    fallback when NVML cannot be read."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -118,7 +119,6 @@ class ClockSampler:
             self.proc.kill()
         self.t.join(timeout=2)
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
@@ -128,12 +128,95 @@ class ClockSampler:
                 mx = float(f[2])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(ClockSampler.NAMES, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvidia-smi every 100 ms over the measurement"}
+
+
+class ClockSampler:
+    """SM clock and throttle reasons of this GPU during the timed regions.  NVML is read
+    (queries only) every millisecond by a thread inside each window, plus one sample
+    at each window edge; when NVML cannot be opened, nvidia-smi samples the whole
+    measurement instead."""
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    BITS = {"hw_slowdown": ("nvmlClocksEventReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": ("nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": ("nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": ("nvmlClocksEventReasonSwPowerCap", 0x4)}
+
+    def __init__(self, uuid):
+        self.sm, self.mx, self.reasons = [], None, set()
+        self._nv = self._h = self._smi = self._thr = self._stop = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.mx = float(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+            self._get_reasons = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                                 or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+            self._bits = {n: int(getattr(pynvml, a, b)) for n, (a, b) in self.BITS.items()}
+            self._nv = pynvml
+        except Exception:
+            self._nv = None
+            self._smi = SmiSampler(uuid)
+
+    def begin(self):
+        if self._smi is not None:
+            self._smi.start()
+
+    def _sample(self):
+        nv, h = self._nv, self._h
+        self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+        r = int(self._get_reasons(h))
+        for n, b in self._bits.items():
+            if r & b:
+                self.reasons.add(n)
+
+    def _poll(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            self._stop.wait(0.001)
+
+    def window_start(self):
+        if self._nv is None:
+            return
+        try:
+            self._sample()
+        except Exception:
+            return
+        self._stop = threading.Event()
+        self._thr = threading.Thread(target=self._poll, daemon=True)
+        self._thr.start()
+
+    def window_stop(self):
+        if self._nv is None or self._thr is None:
+            return
+        self._stop.set()
+        self._thr.join(timeout=2)
+        self._thr = None
+        try:
+            self._sample()
+        except Exception:
+            pass
+
+    def end(self):
+        if self._smi is not None:
+            return self._smi.stop()
+        try:
+            self._nv.nvmlShutdown()
+        except Exception:
+            pass
+        if not self.sm:
+            return None
+        return {"sm_mhz": statistics.median(self.sm), "sm_max_mhz": self.mx, "reasons": sorted(self.reasons),
+                "samples": len(self.sm), "source": "NVML every 1 ms inside the timed regions"}
 
 
 def dist_setup(n_gpus):
@@ -252,9 +335,10 @@ class Workload:
         return n
 
 
-def time_graph(fn, steps, warmup, world):
+def time_graph(fn, steps, warmup, world, clock=None):
     """Capture fn() into a CUDA graph, replay `warmup` times, then time `steps` replays
-    with CUDA events on the capturing stream.  Returns (ms per step, launches per step)."""
+    with CUDA events on the capturing stream (the clock sampler, if any, samples that
+    window).  Returns (ms per step, launches per step)."""
     import torch
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
@@ -271,12 +355,16 @@ def time_graph(fn, steps, warmup, world):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    if clock is not None:
+        clock.window_start()
     with torch.cuda.stream(s):
         e0.record(s)
         for _ in range(steps):
             g.replay()
         e1.record(s)
     torch.cuda.synchronize()
+    if clock is not None:
+        clock.window_stop()
     ms = e0.elapsed_time(e1) / steps
     barrier(world)
     del g
@@ -646,10 +734,10 @@ def run_ours(args):
         gpu_id = str(torch.cuda.current_device())
     clk = ClockSampler(gpu_id) if rank == 0 and not args.no_clocks else None
     if clk:
-        clk.start()
-    ms_step, launches = time_graph(lambda: wl.step(True, True), args.steps, args.warmup, world)
-    ms_gemm, n_gemm = time_graph(lambda: wl.step(False, True), args.steps, args.warmup, world)
-    clocks = clk.stop() if clk else None
+        clk.begin()
+    ms_step, launches = time_graph(lambda: wl.step(True, True), args.steps, args.warmup, world, clk)
+    ms_gemm, n_gemm = time_graph(lambda: wl.step(False, True), args.steps, args.warmup, world, clk)
+    clocks = clk.end() if clk else None
     ms_step = max_over_ranks(world, ms_step)
     ms_gemm = max_over_ranks(world, ms_gemm)
 
