@@ -77,7 +77,10 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 
 /* ---- GEMM variant word -----------------------------------------------------------
  * 0 (W8_VARIANT_AUTO) lets the library choose from its per-shape table (loaded with
- * w8_load_table) or, when the shape is not in it, from a built-in rule.  An explicit
+ * w8_load_table) or, when the shape is not in it, from a built-in rule: Swap-AB with
+ * the balanced partition and a token tile of 16 / 32 / 64 up to 16 / 32 / 64 tokens;
+ * past 64 tokens W8_V_PAIR tiles for FP8-dynamic and INT8, and the 64-wide balanced
+ * Standard loop for Block-FP8.  An explicit
  * variant sets W8_V_EXPLICIT plus:
  *   W8_V_SWAP_AB  compute out^T = W . Aq^T: the 128-row MMA slot runs over N and the
  *                 narrow slot over tokens (the Swap-AB variant, for small M);

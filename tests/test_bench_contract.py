@@ -40,3 +40,14 @@ def test_reference_arm_other_ranks_print_nothing():
                   {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert p.returncode == 0, p.stderr[-2000:]
     assert not [ln for ln in p.stdout.splitlines() if ln.strip().startswith("{")]
+
+
+def test_our_arm_fails_loudly_without_a_gpu():
+    """No CPU fallback: without a device the bench's own arm exits non-zero and prints no
+    result line."""
+    import torch
+    if torch.cuda.is_available():
+        return
+    p = run_bench(["--steps", "3", "--warmup", "3", "--no-cpu"])
+    assert p.returncode != 0
+    assert not [ln for ln in p.stdout.splitlines() if ln.strip().startswith("{")]
