@@ -171,19 +171,60 @@ def _need(t, dtype, name):
         raise TypeError("%s must be a CUDA %s tensor (got %s on %s)" % (name, dtype, t.dtype, t.device))
 
 
+def _dense(t, name, dtype=None, numel=None, shape=None, codes=False):
+    """t must be contiguous (row-major): the C entry points take bare pointers and
+    assume that layout.  codes: any 1-byte element type (e4m3, int8 or raw
+    bytes)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a tensor" % name)
+    if codes and t.element_size() != 1:
+        raise TypeError("%s must hold 1-byte codes (got %s)" % (name, t.dtype))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s (got %s)" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous (row-major)" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s (got %s)" % (name, tuple(shape), tuple(t.shape)))
+    if numel is not None and t.numel() != numel:
+        raise ValueError("%s must have %d elements (got %d)" % (name, numel, t.numel()))
+
+
+def _rows(t, name, dtype):
+    """2-D tensor with unit column stride (its row stride is passed along)."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype:
+        raise TypeError("%s must be a %s tensor" % (name, dtype))
+    if t.dim() != 2 or t.stride(1) != 1 or t.stride(0) < t.shape[1]:
+        raise ValueError("%s must be 2-D with unit column stride" % name)
+
+
+def _cuda(**tensors):
+    """After the layout checks: every tensor argument lives on the GPU."""
+    for name, t in tensors.items():
+        if not t.is_cuda:
+            raise TypeError("%s must be a CUDA tensor (got %s)" % (name, t.device))
+
+
+def _scale_counts(fmt, M, N, K):
+    """Elements of the activation and weight scale arrays of a GEMM in format fmt."""
+    if fmt >= W8_FMT_BLOCK_FP8:
+        return M * (K // 128), ((N + 127) // 128) * (K // 128)
+    return M, N
+
+
 # ---------------------------------------------------------------------------- quantizers
 
 def w8_quant_per_token(x, qfmt=W8_Q_FP8, group=0, ue8m0=False, q=None, scale=None, stream=None):
     """bf16 x[M, K] (row stride x.stride(0)) -> (codes[M, K], scales [M] or [M, K/group])."""
-    _need(x, torch.bfloat16, "x")
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise ValueError("x must be 2-D with unit column stride")
+    _rows(x, "x", torch.bfloat16)
     M, K = x.shape
     qdt = torch.float8_e4m3fn if qfmt == W8_Q_FP8 else torch.int8
     if q is None:
         q = torch.empty((M, K), dtype=qdt, device=x.device)
     if scale is None:
         scale = torch.empty((M,) if group == 0 else (M, K // group), dtype=torch.float32, device=x.device)
+    _dense(q, "q", numel=M * K, codes=True)
+    _dense(scale, "scale", torch.float32, numel=M if group == 0 else M * (K // group))
+    _cuda(x=x, q=q, scale=scale)
     rc = lib().w8_quant_per_token(qfmt, _ptr(x), M, K, x.stride(0), _ptr(q), _ptr(scale), group, int(bool(ue8m0)),
                                   _stream(stream))
     _check("w8_quant_per_token", rc)
@@ -198,6 +239,9 @@ def w8_quant_weight_block(w, ue8m0=False, q=None, scale=None, stream=None):
         q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
     if scale is None:
         scale = torch.empty(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=w.device)
+    _dense(q, "q", numel=N * K, codes=True)
+    _dense(scale, "scale", torch.float32, numel=((N + 127) // 128) * ((K + 127) // 128))
+    _cuda(w=w, q=q, scale=scale)
     rc = lib().w8_quant_weight_block(_ptr(w.contiguous()), N, K, _ptr(q), _ptr(scale), int(bool(ue8m0)),
                                      _stream(stream))
     _check("w8_quant_weight_block", rc)
@@ -205,13 +249,16 @@ def w8_quant_weight_block(w, ue8m0=False, q=None, scale=None, stream=None):
 
 
 def w8_rmsnorm_quant(x, gamma, eps=1e-6, q=None, scale=None, stream=None):
-    _need(x, torch.bfloat16, "x")
-    _need(gamma, torch.bfloat16, "gamma")
+    _rows(x, "x", torch.bfloat16)
     M, H = x.shape
+    _dense(gamma, "gamma", torch.bfloat16, numel=H)
     if q is None:
         q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
     if scale is None:
         scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _dense(q, "q", numel=M * H, codes=True)
+    _dense(scale, "scale", torch.float32, numel=M)
+    _cuda(x=x, gamma=gamma, q=q, scale=scale)
     rc = lib().w8_rmsnorm_quant(_ptr(x), _ptr(gamma), float(eps), M, H, x.stride(0), _ptr(q), _ptr(scale),
                                 _stream(stream))
     _check("w8_rmsnorm_quant", rc)
@@ -220,13 +267,18 @@ def w8_rmsnorm_quant(x, gamma, eps=1e-6, q=None, scale=None, stream=None):
 
 def w8_silu_mul_quant(gate_up, q=None, scale=None, stream=None):
     """bf16 gate_up[M, 2I] (gate first) -> (e4m3 codes of silu(gate)*up [M, I], scales [M])."""
-    _need(gate_up, torch.bfloat16, "gate_up")
+    _rows(gate_up, "gate_up", torch.bfloat16)
     M, I2 = gate_up.shape
+    if I2 % 2:
+        raise ValueError("gate_up must have an even number of columns [gate | up]")
     I = I2 // 2
     if q is None:
         q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=gate_up.device)
     if scale is None:
         scale = torch.empty((M,), dtype=torch.float32, device=gate_up.device)
+    _dense(q, "q", numel=M * I, codes=True)
+    _dense(scale, "scale", torch.float32, numel=M)
+    _cuda(gate_up=gate_up, q=q, scale=scale)
     rc = lib().w8_silu_mul_quant(_ptr(gate_up), M, I, gate_up.stride(0), _ptr(q), _ptr(scale), _stream(stream))
     _check("w8_silu_mul_quant", rc)
     return q, scale
@@ -234,13 +286,16 @@ def w8_silu_mul_quant(gate_up, q=None, scale=None, stream=None):
 
 def w8_rmsnorm_quant_group(x, gamma, eps=1e-6, group=128, ue8m0=False, q=None, scale=None, stream=None):
     """rms_norm + 1x128-group fp8 quant: (e4m3 codes [M, H], scales [M, H/group])."""
-    _need(x, torch.bfloat16, "x")
-    _need(gamma, torch.bfloat16, "gamma")
+    _rows(x, "x", torch.bfloat16)
     M, H = x.shape
+    _dense(gamma, "gamma", torch.bfloat16, numel=H)
     if q is None:
         q = torch.empty((M, H), dtype=torch.float8_e4m3fn, device=x.device)
     if scale is None:
         scale = torch.empty((M, H // group), dtype=torch.float32, device=x.device)
+    _dense(q, "q", numel=M * H, codes=True)
+    _dense(scale, "scale", torch.float32, numel=M * (H // group))
+    _cuda(x=x, gamma=gamma, q=q, scale=scale)
     rc = lib().w8_rmsnorm_quant_group(_ptr(x), _ptr(gamma), float(eps), M, H, x.stride(0), group, int(bool(ue8m0)),
                                       _ptr(q), _ptr(scale), _stream(stream))
     _check("w8_rmsnorm_quant_group", rc)
@@ -249,13 +304,18 @@ def w8_rmsnorm_quant_group(x, gamma, eps=1e-6, group=128, ue8m0=False, q=None, s
 
 def w8_silu_mul_quant_group(gate_up, group=128, ue8m0=False, q=None, scale=None, stream=None):
     """silu_and_mul + 1x128-group fp8 quant: (e4m3 codes [M, I], scales [M, I/group])."""
-    _need(gate_up, torch.bfloat16, "gate_up")
+    _rows(gate_up, "gate_up", torch.bfloat16)
     M, I2 = gate_up.shape
+    if I2 % 2:
+        raise ValueError("gate_up must have an even number of columns [gate | up]")
     I = I2 // 2
     if q is None:
         q = torch.empty((M, I), dtype=torch.float8_e4m3fn, device=gate_up.device)
     if scale is None:
         scale = torch.empty((M, I // group), dtype=torch.float32, device=gate_up.device)
+    _dense(q, "q", numel=M * I, codes=True)
+    _dense(scale, "scale", torch.float32, numel=M * (I // group))
+    _cuda(gate_up=gate_up, q=q, scale=scale)
     rc = lib().w8_silu_mul_quant_group(_ptr(gate_up), M, I, gate_up.stride(0), group, int(bool(ue8m0)), _ptr(q),
                                        _ptr(scale), _stream(stream))
     _check("w8_silu_mul_quant_group", rc)
@@ -319,13 +379,19 @@ def _workspace(ws, device, nbytes):
 
 def w8_gemm(fmt, A_q, A_scale, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
     """out[M, N] (bf16) = scaled A_q . W_q^T in format `fmt` (W8_FMT_*)."""
+    _dense(A_q, "A_q", codes=True)
+    _dense(W_q, "W_q", codes=True)
+    if A_q.dim() != 2 or W_q.dim() != 2 or W_q.shape[1] != A_q.shape[1]:
+        raise ValueError("A_q [M, K] and W_q [N, K] expected")
     M, K = A_q.shape
     N = W_q.shape[0]
-    if W_q.shape[1] != K:
-        raise ValueError("K mismatch")
+    na, nw = _scale_counts(fmt, M, N, K)
+    _dense(A_scale, "A_scale", torch.float32, numel=na)
+    _dense(W_scale, "W_scale", torch.float32, numel=nw)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A_q.device)
-    _need(out, torch.bfloat16, "out")
+    _dense(out, "out", torch.bfloat16, shape=(M, N))
+    _cuda(A_q=A_q, A_scale=A_scale, W_q=W_q, W_scale=W_scale, out=out)
     nbytes = w8_gemm_workspace_size(fmt, M, N, K, variant)
     wp, wn = _workspace(workspace, A_q.device, nbytes)
     rc = lib().w8_gemm(fmt, _ptr(A_q), _ptr(A_scale), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp, wn,
@@ -346,16 +412,22 @@ def w8_grouped_gemm(fmt, A_q, A_scale, W_q, W_scale, expert_offsets, max_tokens_
     """Mixture-of-experts GEMM: A_q [T, K] rows sorted by expert (rows [off[e], off[e+1])
     belong to expert e), W_q [E, N, K], W_scale [E, N]; expert_offsets int32 [E+1] on the
     device.  Rows no expert owns are left as they were in `out`."""
+    _dense(A_q, "A_q", codes=True)
+    _dense(W_q, "W_q", codes=True)
+    if A_q.dim() != 2 or W_q.dim() != 3 or W_q.shape[2] != A_q.shape[1]:
+        raise ValueError("A_q [T, K] and W_q [E, N, K] expected")
     T, K = A_q.shape
-    E, N, K2 = W_q.shape
-    if K2 != K:
-        raise ValueError("K mismatch")
+    E, N, _ = W_q.shape
     if expert_offsets.dtype != torch.int32 or not expert_offsets.is_cuda or expert_offsets.numel() != E + 1:
         raise TypeError("expert_offsets must be a CUDA int32 tensor of E + 1 entries")
+    _dense(expert_offsets, "expert_offsets", torch.int32)
+    _dense(A_scale, "A_scale", torch.float32, numel=T)
+    _dense(W_scale, "W_scale", torch.float32, numel=E * N)
     mm = T if max_tokens_per_expert is None else int(max_tokens_per_expert)
     if out is None:
         out = torch.zeros((T, N), dtype=torch.bfloat16, device=A_q.device)
-    _need(out, torch.bfloat16, "out")
+    _dense(out, "out", torch.bfloat16, shape=(T, N))
+    _cuda(A_q=A_q, A_scale=A_scale, W_q=W_q, W_scale=W_scale, out=out, expert_offsets=expert_offsets)
     nbytes = w8_grouped_gemm_workspace_size(fmt, E, T, N, K, mm, variant)
     wp, wn = _workspace(workspace, A_q.device, nbytes)
     rc = lib().w8_grouped_gemm(fmt, _ptr(A_q), _ptr(A_scale), _ptr(W_q), _ptr(W_scale), _ptr(out),
@@ -373,11 +445,14 @@ def w8_qk_norm_rope(qkv, Hq, Hkv, D, q_weight, k_weight, cos_sin, positions, eps
         raise ValueError("qkv must be contiguous [T, (Hq + 2 Hkv) * D]")
     if out is None:
         out = torch.empty_like(qkv)
-    _need(out, torch.bfloat16, "out")
-    _need(q_weight, torch.bfloat16, "q_weight")
-    _need(k_weight, torch.bfloat16, "k_weight")
-    _need(cos_sin, torch.float32, "cos_sin")
-    _need(positions, torch.int64, "positions")
+    _dense(out, "out", torch.bfloat16, shape=tuple(qkv.shape))
+    _dense(q_weight, "q_weight", torch.bfloat16, numel=D)
+    _dense(k_weight, "k_weight", torch.bfloat16, numel=D)
+    _dense(cos_sin, "cos_sin", torch.float32)
+    if cos_sin.dim() != 2 or cos_sin.shape[1] != D:
+        raise ValueError("cos_sin must be [max_pos, D]")
+    _dense(positions, "positions", torch.int64, numel=T)
+    _cuda(qkv=qkv, out=out, q_weight=q_weight, k_weight=k_weight, cos_sin=cos_sin, positions=positions)
     rc = lib().w8_qk_norm_rope(_ptr(qkv), _ptr(out), T, Hq, Hkv, D, _ptr(q_weight), _ptr(k_weight), _ptr(cos_sin),
                                cos_sin.shape[0], _ptr(positions), float(eps), _stream(stream))
     _check("w8_qk_norm_rope", rc)
@@ -403,14 +478,17 @@ def w8_linear(fmt, x, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace
     """out[M, N] (bf16) = scaled quant(x) . W_q^T: x bf16 [M, K] quantized per token (or
     per 1 x 128 group for Block-FP8) and multiplied in one call: the quantizer and the
     GEMM, or one kernel when the variant carries W8_V_FUSED."""
-    _need(x, torch.bfloat16, "x")
+    _rows(x, "x", torch.bfloat16)
     M, K = x.shape
+    _dense(W_q, "W_q", codes=True)
+    if W_q.dim() != 2 or W_q.shape[1] != K:
+        raise ValueError("W_q [N, K] expected")
     N = W_q.shape[0]
-    if W_q.shape[1] != K:
-        raise ValueError("K mismatch")
+    _dense(W_scale, "W_scale", torch.float32, numel=_scale_counts(fmt, M, N, K)[1])
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
-    _need(out, torch.bfloat16, "out")
+    _dense(out, "out", torch.bfloat16, shape=(M, N))
+    _cuda(x=x, W_q=W_q, W_scale=W_scale, out=out)
     nbytes = w8_linear_workspace_size(fmt, M, N, K, variant)
     wp, wn = _workspace(workspace, x.device, nbytes)
     rc = lib().w8_linear(fmt, _ptr(x), x.stride(0), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp, wn,
@@ -421,12 +499,17 @@ def w8_linear(fmt, x, W_q, W_scale, out=None, variant=W8_VARIANT_AUTO, workspace
 
 def w8_linear_debug(fmt, x, W_q, W_scale, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
     """One-kernel w8_linear that also returns the codes [M, K] (uint8) and scales it computed."""
-    _need(x, torch.bfloat16, "x")
+    _rows(x, "x", torch.bfloat16)
     M, K = x.shape
+    _dense(W_q, "W_q", codes=True)
+    if W_q.dim() != 2 or W_q.shape[1] != K:
+        raise ValueError("W_q [N, K] expected")
     N = W_q.shape[0]
+    _dense(W_scale, "W_scale", torch.float32, numel=_scale_counts(fmt, M, N, K)[1])
     out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     q = torch.zeros((M, K), dtype=torch.uint8, device=x.device)
     s = torch.zeros((M, K // 128) if fmt >= W8_FMT_BLOCK_FP8 else (M,), dtype=torch.float32, device=x.device)
+    _cuda(x=x, W_q=W_q, W_scale=W_scale)
     nbytes = w8_linear_workspace_size(fmt, M, N, K, variant)
     wp, wn = _workspace(workspace, x.device, nbytes)
     rc = lib().w8_linear_debug(fmt, _ptr(x), x.stride(0), _ptr(W_q), _ptr(W_scale), _ptr(out), M, N, K, variant, wp,
@@ -437,10 +520,16 @@ def w8_linear_debug(fmt, x, W_q, W_scale, variant=W8_VARIANT_AUTO, workspace=Non
 
 def w8_gemm_i32_debug(A_q, W_q, acc=None, variant=W8_VARIANT_AUTO, workspace=None, stream=None):
     """Raw int32 accumulators acc[M, N] = sum_k A_q W_q (INT8 path, no scales)."""
+    _dense(A_q, "A_q", codes=True)
+    _dense(W_q, "W_q", codes=True)
+    if A_q.dim() != 2 or W_q.dim() != 2 or W_q.shape[1] != A_q.shape[1]:
+        raise ValueError("A_q [M, K] and W_q [N, K] expected")
     M, K = A_q.shape
     N = W_q.shape[0]
     if acc is None:
         acc = torch.empty((M, N), dtype=torch.int32, device=A_q.device)
+    _dense(acc, "acc", torch.int32, shape=(M, N))
+    _cuda(A_q=A_q, W_q=W_q, acc=acc)
     nbytes = w8_gemm_workspace_size(W8_FMT_INT8, M, N, K, variant)
     wp, wn = _workspace(workspace, A_q.device, nbytes)
     rc = lib().w8_gemm_i32_debug(_ptr(A_q), _ptr(W_q), _ptr(acc), M, N, K, variant, wp, wn, _stream(stream))
