@@ -22,7 +22,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = build_oracle.build()
+        # W8_ORACLE_LIB: another build of the same C source (the mutation test loads
+        # copies with a planted mistake this way)
+        path = os.environ.get("W8_ORACLE_LIB") or build_oracle.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i, f = ctypes.c_int, ctypes.c_float
