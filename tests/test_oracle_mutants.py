@@ -2,10 +2,12 @@
 dropped term, a wrong sign, index or constant, a transposed operand, a wrong rounding)
 into a copy of the C oracle, builds it with the same compiler flags, and runs the
 oracle's pin tests against that build (W8_ORACLE_LIB): at least one pin must fail.  The
-unmodified copy, built the same way, must pass them all.  The mistakes keep every
+unmodified copy, built the same way, must pass them all.  Mistakes in the Python front
+end (the grouped GEMM) are planted in a copy of the package imported ahead of it.  The mistakes keep every
 access in bounds, so a mutant fails by assertion, never by a crash."""
 import concurrent.futures
 import os
+import shutil
 import subprocess
 import sys
 
@@ -112,6 +114,21 @@ MUTANTS = [
 ]
 
 
+# the same for the oracle's Python front end (a mutated copy of the package, imported
+# ahead of the original)
+PY_MUTANTS = [
+    ("grouped GEMM takes the next expert's weights",
+     "np.asarray(Wq)[e], np.asarray(sW)[e])",
+     "np.asarray(Wq)[(e + 1) % E], np.asarray(sW)[e])"),
+    ("grouped GEMM uses the first expert's scales",
+     "np.asarray(Wq)[e], np.asarray(sW)[e])",
+     "np.asarray(Wq)[e], np.asarray(sW)[0])"),
+    ("grouped GEMM does not slice the token scales",
+     "np.asarray(sA)[lo:hi]",
+     "np.asarray(sA)[:hi - lo]"),
+]
+
+
 def _build(src_text, path):
     c = path + ".c"
     with open(c, "w") as fh:
@@ -121,11 +138,29 @@ def _build(src_text, path):
     return path
 
 
-def _pins(lib, files):
+def _pins(lib, files, pkg_dir=None):
     env = dict(os.environ, W8_ORACLE_LIB=lib)
-    p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", "-m", "not gpu"] + files,
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    cwd = ROOT
+    if pkg_dir is not None:
+        # the copy first on the path (and not the working directory, which would put the
+        # original first)
+        env["PYTHONPATH"] = os.pathsep.join([pkg_dir, ROOT])
+        cwd = pkg_dir
+    p = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", "-m", "not gpu",
+                        "--rootdir", ROOT] + [os.path.join(ROOT, f) for f in files],
+                       cwd=cwd, env=env, capture_output=True, text=True, timeout=600)
     return p.returncode, p.stdout[-1500:]
+
+
+def _py_copy(text, path):
+    """A copy of the oracle package whose oracle.py is `text`."""
+    pkg = os.path.join(path, "oracle")
+    os.makedirs(pkg)
+    for f in ("__init__.py", "build_oracle.py", "w8_oracle.c"):
+        shutil.copy2(os.path.join(ROOT, "oracle", f), pkg)
+    with open(os.path.join(pkg, "oracle.py"), "w") as fh:
+        fh.write(text)
+    return path
 
 
 def test_planted_mistakes_fail_a_pin(tmp_path):
@@ -135,11 +170,24 @@ def test_planted_mistakes_fail_a_pin(tmp_path):
         assert src.count(old) == 1, "planting site not found (oracle edited?): %s" % name
         jobs.append((name, src.replace(old, new), PINS[group], False))
 
+    py_src = open(os.path.join(ROOT, "oracle", "oracle.py")).read()
+    py_jobs = [("unmodified Python front end", py_src, True)]
+    for name, old, new in PY_MUTANTS:
+        assert py_src.count(old) == 1, "planting site not found (oracle edited?): %s" % name
+        py_jobs.append((name, py_src.replace(old, new), False))
+    clean_lib = _build(src, str(tmp_path / "clean.so"))
+
     def run(job):
         name, text, files, clean = job
-        lib = _build(text, str(tmp_path / ("m%d.so" % abs(hash(name)))))
-        rc, out = _pins(lib, files)
+        if files is None:      # Python front-end mutant, on the unmodified C library
+            d = _py_copy(text, str(tmp_path / ("p%d" % abs(hash(name)))))
+            rc, out = _pins(clean_lib, PINS["gemm"], d)
+        else:
+            lib = _build(text, str(tmp_path / ("m%d.so" % abs(hash(name)))))
+            rc, out = _pins(lib, files)
         return name, clean, rc, out
+
+    jobs += [(name, text, None, clean) for name, text, clean in py_jobs]
 
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         results = list(ex.map(run, jobs))
@@ -148,7 +196,12 @@ def test_planted_mistakes_fail_a_pin(tmp_path):
         if clean:
             if rc != 0:
                 broken.append((name, rc, out))
-        elif rc != 1:          # 1: some test failed (0: all passed; other: crash / collection error)
-            survivors.append((name, rc, out))
+        else:
+            # caught = a pin failed on an assertion: exit status 1 and a summary line with
+            # "failed" and no "error" (0: all passed; other statuses: a crash or a
+            # collection error, which would not show that a pin catches the mistake)
+            summary = out.strip().splitlines()[-1] if out.strip() else ""
+            if rc != 1 or "failed" not in summary or "error" in summary:
+                survivors.append((name, rc, out))
     assert not broken, broken
     assert not survivors, survivors
