@@ -793,7 +793,9 @@ def run_ours(args):
         out["e2e"] = e2e
     if detail:
         out["detail"] = detail
-    if rank == 0 and not args.no_extras:
+    # single-GPU timings of the other kernels: at N = 1 only (with more ranks the others
+    # would sit idle, holding their GPUs, while rank 0 times them)
+    if rank == 0 and world == 1 and not args.no_extras:
         out["other_kernels"] = time_extras(dev, peak)
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(shapes, ms, target_s=args.cpu_seconds)
