@@ -46,6 +46,8 @@ def lib():
         L.orc_quant_rows.restype = i
         L.orc_quant_weight_block.argtypes = [P, i, i, P, P, i]
         L.orc_quant_weight_block.restype = i
+        L.orc_sumsq_f32.argtypes = [P, i]
+        L.orc_sumsq_f32.restype = f
         L.orc_rmsnorm_f32.argtypes = [P, P, f, i, i, i, P]
         L.orc_rmsnorm_f32.restype = None
         L.orc_rmsnorm_quant.argtypes = [P, P, f, i, i, i, P, P]
@@ -144,6 +146,13 @@ def quant_weight_block(w_bits, ue8m0=False):
     s = np.zeros(((N + 127) // 128, (K + 127) // 128), dtype=np.float32)
     lib().orc_quant_weight_block(_p(w), N, K, _p(q), _p(s), int(bool(ue8m0)))
     return q, s
+
+
+def sumsq_f32(x_bits):
+    """fp32 rounding (to nearest, ties to even) of the exact sum of squares of a 1-D
+    array of bf16 values (raw bits)."""
+    x = _c(x_bits, np.uint16).reshape(-1)
+    return np.float32(lib().orc_sumsq_f32(_p(x), int(x.size)))
 
 
 def rmsnorm_f32(x_bits, gamma_bits, eps):

@@ -209,10 +209,65 @@ int orc_quant_weight_block(const uint16_t* w, int N, int K, uint8_t* q, float* s
 /* Fused producers                                                            */
 /* ------------------------------------------------------------------------- */
 
+/* Sum of squares of n bf16 values, exactly, then rounded once to fp32 (round to
+ * nearest, ties to even).  The pages fix no summation order, so the sum is taken as
+ * the mathematical one: its fp32 rounding is then a function of the values alone.
+ *
+ * Each finite bf16 is q * 2^e with an integer q < 256 (8 significant bits) and
+ * e >= -133, so each square is q^2 * 2^(2e), an integer q^2 < 2^16 times a power of two
+ * no smaller than 2^-266.  The sum is accumulated as an exact integer count of units
+ * of 2^-266 in a 576-bit number (18 words of 32 bits; the largest square of a finite
+ * bf16 needs bit 506 and a sum of up to 2^31 of them at most 31 bits more), then
+ * rounded to fp32 by inspecting its bits.  Any NaN input gives NaN, any infinity +inf. */
+#define ORC_SQ_WORDS 18
+float orc_sumsq_f32(const uint16_t* x, int n)
+{
+    uint32_t acc[ORC_SQ_WORDS];
+    memset(acc, 0, sizeof acc);
+    int has_nan = 0, has_inf = 0;
+    for (int k = 0; k < n; ++k) {
+        const unsigned E = (x[k] >> 7) & 0xFFu, m = x[k] & 0x7Fu;
+        if (E == 0xFFu) {
+            if (m) has_nan = 1; else has_inf = 1;
+            continue;
+        }
+        const uint64_t q = (E == 0) ? m : (128u + m);         /* |x| = q * 2^e */
+        const int e = (E == 0) ? -133 : (int)E - 134;
+        const int shift = 2 * e + 266;                        /* x^2 = q^2 * 2^shift units */
+        int w = shift / 32;
+        uint64_t add = (q * q) << (shift % 32);               /* < 2^48: two words */
+        while (add != 0 && w < ORC_SQ_WORDS) {
+            const uint64_t t = (uint64_t)acc[w] + (add & 0xFFFFFFFFu);
+            acc[w] = (uint32_t)t;
+            add = (add >> 32) + (t >> 32);
+            ++w;
+        }
+    }
+    if (has_nan) return NAN;
+    if (has_inf) return INFINITY;
+    /* highest set bit p: the sum lies in [2^(p-266), 2^(p-265)) */
+    int p = -1;
+    for (int w = ORC_SQ_WORDS - 1; w >= 0 && p < 0; --w)
+        for (int b = 31; b >= 0; --b)
+            if ((acc[w] >> b) & 1u) { p = 32 * w + b; break; }
+    if (p < 0) return 0.0f;
+    /* fp32 keeps 24 bits from p down, and nothing below 2^-149 (bit 117 here) */
+    int lsb = p - 23;
+    if (lsb < 117) lsb = 117;
+#define ORC_SQ_BIT(i) ((acc[(i) / 32] >> ((i) % 32)) & 1u)
+    uint32_t mant = 0;
+    for (int i = p; i >= lsb; --i) mant = (mant << 1) | ORC_SQ_BIT(i);
+    const unsigned half = ORC_SQ_BIT(lsb - 1);
+    unsigned sticky = 0;
+    for (int i = lsb - 2; i >= 0 && !sticky; --i) sticky = ORC_SQ_BIT(i);
+#undef ORC_SQ_BIT
+    if (half && (sticky || (mant & 1u))) ++mant;             /* ties to even */
+    return ldexpf((float)mant, lsb - 266);                   /* exact, or +inf past FLT_MAX */
+}
+
 /* RMS normalization in fp32 ([FP8] "Patron de fusion del forward pass":
  * post-attention rms_norm fused with the per-token fp8 quant):
- *   ss   = sum_k x_k^2, accumulated in fp64 (each square of a bf16 is exact in fp64),
- *          then rounded once to fp32;
+ *   ss   = sum_k x_k^2, the exact sum rounded once to fp32 (orc_sumsq_f32);
  *   mean = ss / H;  r = 1 / sqrt(mean + eps)    (fp32, each step correctly rounded);
  *   y_k  = (x_k * r) * gamma_k                  (fp32, in this order).
  * y stays fp32 (the point of the fusion: no bf16 round trip before the quant). */
@@ -221,12 +276,8 @@ void orc_rmsnorm_f32(const uint16_t* x, const uint16_t* gamma, float eps,
 {
     for (int m = 0; m < M; ++m) {
         const uint16_t* xr = x + (size_t)m * ldx;
-        double ss = 0.0;
-        for (int k = 0; k < H; ++k) {
-            double xv = (double)orc_bf16_to_float(xr[k]);
-            ss += xv * xv;
-        }
-        float mean = (float)ss / (float)H;
+        float ss = orc_sumsq_f32(xr, H);
+        float mean = ss / (float)H;
         float r = 1.0f / sqrtf(mean + eps);
         for (int k = 0; k < H; ++k)
             y[(size_t)m * H + k] = (orc_bf16_to_float(xr[k]) * r) * orc_bf16_to_float(gamma[k]);
@@ -546,7 +597,7 @@ int orc_gemm_split_k(int fmt, const uint8_t* Aq, const float* sA, const uint8_t*
  * query heads, then the Hkv key heads, then the Hkv value heads, D values each):
  *   for every token t and every query or key head (x = that head's D values):
  *     y = rms_norm of x with the head-dimension weight (q_weight for query heads,
- *         k_weight for key heads): fp64 sum of squares rounded once to fp32, then
+ *         k_weight for key heads): the exact sum of squares rounded once to fp32, then
  *         mean = ss / D, r = 1 / sqrt(mean + eps), y_k = (x_k * r) * w_k in fp32;
  *     with p = positions[t], c_i = cos_sin[p * D + i] and s_i = cos_sin[p * D + D/2 + i]
  *     (i < D/2), each pair (y_i, y_{i+D/2}) is rotated by the angle whose cosine and
@@ -578,12 +629,8 @@ int orc_qk_norm_rope(const uint16_t* qkv, uint16_t* out, int T, int Hq, int Hkv,
                 continue;
             }
             const uint16_t* w = (h < Hq) ? q_weight : k_weight;
-            double ss = 0.0;
-            for (int k = 0; k < D; ++k) {
-                double xv = (double)orc_bf16_to_float(x[k]);
-                ss += xv * xv;
-            }
-            float mean = (float)ss / (float)D;
+            float ss = orc_sumsq_f32(x, D);
+            float mean = ss / (float)D;
             float r = 1.0f / sqrtf(mean + eps);
             for (int k = 0; k < D; ++k) y[k] = (orc_bf16_to_float(x[k]) * r) * orc_bf16_to_float(w[k]);
             for (int i = 0; i < half; ++i) {

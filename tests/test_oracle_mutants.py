@@ -18,6 +18,7 @@ PINS = {
     "quant": ["tests/test_oracle_quant.py"],
     "gemm": ["tests/test_oracle_gemm.py", "tests/test_oracle_grouped.py"],
     "qknr": ["tests/test_oracle_qknr.py"],
+    "sumsq": ["tests/test_oracle_sumsq.py"],
 }
 
 # (name, text of the oracle, planted replacement, pin files that must catch it)
@@ -62,8 +63,23 @@ MUTANTS = [
      "        float r = 1.0f / sqrtf(mean + eps);\n        for (int k = 0; k < H; ++k)",
      "        float r = 1.0f / sqrtf(mean);\n        for (int k = 0; k < H; ++k)", "quant"),
     ("rms_norm mean over H - 1",
-     "float mean = (float)ss / (float)H;",
-     "float mean = (float)ss / (float)(H - 1);", "quant"),
+     "float mean = ss / (float)H;",
+     "float mean = ss / (float)(H - 1);", "quant"),
+    ("sum of squares drops the sticky bits",
+     "for (int i = lsb - 2; i >= 0 && !sticky; --i) sticky = ORC_SQ_BIT(i);",
+     "for (int i = lsb - 2; i >= lsb - 2 && !sticky; --i) sticky = ORC_SQ_BIT(i);", "sumsq"),
+    ("sum of squares rounds ties up",
+     "if (half && (sticky || (mant & 1u))) ++mant;",
+     "if (half) ++mant;", "sumsq"),
+    ("sum of squares with the exponent of normal values off by one",
+     "const int e = (E == 0) ? -133 : (int)E - 134;",
+     "const int e = (E == 0) ? -133 : (int)E - 133;", "sumsq"),
+    ("sum of squares keeps fp32 subnormals one bit too fine",
+     "if (lsb < 117) lsb = 117;",
+     "if (lsb < 116) lsb = 116;", "sumsq"),
+    ("sum of squares loses the carry between words",
+     "add = (add >> 32) + (t >> 32);",
+     "add = (add >> 32);", "sumsq"),
     ("rms_norm without gamma",
      "y[(size_t)m * H + k] = (orc_bf16_to_float(xr[k]) * r) * orc_bf16_to_float(gamma[k]);",
      "y[(size_t)m * H + k] = orc_bf16_to_float(xr[k]) * r;", "quant"),
