@@ -4,9 +4,14 @@
 // framework whose allocator they do not own (a plugin, a custom operator in a runtime
 // that forbids cudaMalloc while serving), or code that must not allocate at all after
 // start-up (a latency-critical service, a memory budget fixed at load time).  For them
-// w8_gemm_noalloc uses a scratch area that the library itself places in device memory
-// at load time: the file-scope array below.  Every GPU that loads the library holds it
-// until the process exits.
+// w8_gemm_noalloc uses a scratch area that belongs to the library's device code: the
+// file-scope array below.  Every GPU that uses it holds it until the process exits.
+//
+// When the array reaches the device: with eager module loading, when the library's
+// device code is loaded; with lazy module loading (CUDA_MODULE_LOADING=LAZY, the
+// default of recent CUDA releases), when its address is first asked for.  That happens
+// in the first call on each device, whatever variant that call resolves to, so one
+// warm-up call before a memory budget is fixed (or before a stream capture) settles it.
 //
 // The array is shared by every call on a device and keeps what the last call left in
 // it; the ticket counters a call uses are cleared at the start of that call.  Calls
@@ -67,13 +72,17 @@ extern "C" int w8_gemm_noalloc(int fmt, const void* A_q, const float* A_scale, c
     rc = gemm_plan(fmt, M, N, K, v, sms, &plan);
     if (rc != W8_OK) return rc;
     if (plan.ws_bytes > kNoAllocScratchBytes) return W8_ERR_WORKSPACE;   // beyond the fixed maximum
+    // the address is looked up on every device's first call, whether or not this call
+    // needs scratch, so that the array is in place after any first call
     void* scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc != W8_OK) return rc;
     if (plan.ws_bytes > 0) {
-        rc = noalloc_scratch(&scratch);
-        if (rc != W8_OK) return rc;
         // counters of this call's tiles must start at zero
         cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
         if (cudaMemsetAsync(scratch, 0, (size_t)plan.tiles * 4, s) != cudaSuccess) return W8_ERR_CUDA;
+    } else {
+        scratch = nullptr;
     }
     return gemm_launch(plan, A_q, A_scale, W_q, W_scale, out, nullptr, scratch, kNoAllocScratchBytes,
                        reinterpret_cast<cudaStream_t>(stream));
