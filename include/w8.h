@@ -126,6 +126,17 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 accumulator over the whole K range, K blocks in order (INT8
  *                 accumulators are exact).  For prefill sizes; with PDL the kernel waits
  *                 for the kernels ahead before its first load.
+ *   W8_V_DECODE   decode form (M <= 64; FP8-dynamic or INT8; no W8_V_SWAP_AB / W8_V_STREAM /
+ *                 W8_V_CLUSTER / W8_V_BM64 / W8_V_PAIR): the tokens occupy the tensor
+ *                 core's 64-row operand and BN = 16 * (tile + 1) weight rows (64..256) its
+ *                 wide one, so each MMA consumes BN x 32 weight bytes.  The split field
+ *                 holds C - 1: each weight tile's K range is cut into C = 1..8 contiguous
+ *                 chunks (at most one per 128-column K block), run as one thread-block
+ *                 cluster of C CTAs; their fp32 (int32 for INT8) partial sums are added in
+ *                 chunk order in distributed shared memory, each rank finishing a share of
+ *                 the tile's columns.  No workspace.  Stages as above (default 3); bits
+ *                 27..30: K blocks of weights each CTA keeps in flight into L2 ahead of its
+ *                 stages (0 = none).  The variant for decode token counts.
  *   W8_V_PDL      launch with programmatic dependent launch: the kernel may start while
  *                 earlier kernels on the stream still run, and it reads weight tiles
  *                 (into shared memory and L2) before waiting for them.  Only legal when
@@ -146,6 +157,8 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 #define W8_V_PFIX (1 << 19)
 #define W8_V_FUSED (1 << 24)
 #define W8_V_PAIR (1 << 25)
+#define W8_V_DECODE (1 << 26)
+#define W8_V_L2_SHIFT 27
 #define W8_V_KPS_SHIFT 20
 #define W8_V_CPS_SHIFT 22
 #define W8_VARIANT(swap, log2_split, tile, stream)                                            \
@@ -339,15 +352,17 @@ W8_API int w8_linear_debug(int fmt, const void* x, int ldx, const void* W_q, con
  * Split-K workspace because they may not call cudaMalloc -- code running inside a
  * runtime whose allocator it does not own, or a service whose device memory is fixed
  * at start-up.  This entry point takes the same arguments as w8_gemm minus the
- * workspace and uses instead a scratch array the library places in device memory when
- * it is loaded: 8 MiB per GPU, held until the process exits.  A variant whose
- * workspace would exceed that (see w8_gemm_workspace_size) returns W8_ERR_WORKSPACE.
- * It allocates nothing: the first call on each device looks up the array's device
- * address (a runtime query, no allocation); make that first call before any stream
- * capture.  Each call clears the ticket counters it uses with cudaMemsetAsync on
- * `stream`.  All calls on a device share the array, so calls that overlap on the GPU
- * (e.g. on two streams at once) race; successive calls on one stream are fine.
- * Errors: as w8_gemm. */
+ * workspace and uses instead a scratch array that is part of the library's device
+ * code: 8 MiB per GPU, held until the process exits.  A variant whose workspace would
+ * exceed that (see w8_gemm_workspace_size) returns W8_ERR_WORKSPACE.  It calls no
+ * allocator.  The first call on each device looks up the array's device address; with
+ * lazy module loading (CUDA_MODULE_LOADING=LAZY, the default of recent CUDA releases)
+ * that lookup is also when the driver places the array -- and the kernels' code -- on
+ * the device.  So make one call (any shape or variant) before a memory budget is fixed
+ * and before any stream capture.  Each call clears the ticket counters it uses with
+ * cudaMemsetAsync on `stream`.  All calls on a device share the array, so calls that
+ * overlap on the GPU (e.g. on two streams at once) race; successive calls on one
+ * stream are fine.  Errors: as w8_gemm. */
 W8_API int w8_gemm_noalloc(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                            void* out, int M, int N, int K, int variant, w8_stream_t stream);
 
