@@ -3,6 +3,8 @@
 // families (w8_gemm_f8.cu, w8_gemm_i8.cu, w8_gemm_block.cu, w8_gemm_bm64.cu,
 // w8_gemm_fq.cu, w8_gemm_grouped.cu, and the CTA-pair loop of w8_gemm_pair.cu).  The
 // kernel itself and what it computes are described in w8_gemm_kernel.cuh.
+#include <algorithm>
+
 #include "w8_gemm_kernel.cuh"
 
 namespace w8 {
@@ -105,6 +107,76 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
     q.bm = (variant & W8_V_BM64) ? 64 : 128;
     q.pfix = (variant & W8_V_PFIX) ? 1 : 0;
     if (lg > 8) return W8_ERR_UNSUPPORTED;
+    if (variant & W8_V_DECODE) {
+        // decode form (w8_gemm_decode.cu): tokens in the 64-row MMA operand, 16 (tile + 1)
+        // weight rows in the wide one, split + 1 K chunks per weight tile as one cluster
+        if (block || q.swap || q.stream || q.cluster || q.bm != 128 || q.pfix || (variant & W8_V_PAIR) || M > 64)
+            return W8_ERR_UNSUPPORTED;
+        const int bn = 16 * (tid + 1);
+        const int C = lg + 1;
+        if (bn < 64 || C > 8) return W8_ERR_UNSUPPORTED;
+        q.kbs = (K + 127) / 128;
+        if (C > q.kbs) return W8_ERR_UNSUPPORTED;
+        // default depth: about 108 KB of stages, the most that still lets a CTA of the next
+        // GEMM share the SM (bytes in flight per SM are what sets the streaming rate)
+        if (stages == 0) stages = (int)std::max<size_t>(2, std::min<size_t>(8, 110592 / ((size_t)(((M + 7) & ~7) + bn) * 128)));
+        if (stages < 2) return W8_ERR_UNSUPPORTED;
+        q.decode = 1;
+        q.bn = bn;
+        q.split = C;
+        q.kps = 1;
+        q.stages = stages;
+        q.m8 = (M + 7) & ~7;
+        q.l2ahead = (variant >> W8_V_L2_SHIFT) & 0xF;
+        q.sw = ((bn + 16 * C - 1) / (16 * C)) * 16;
+        const size_t stage = (size_t)(q.m8 + bn) * 128;
+        // stages, barriers, TMEM slot and flag, then the scales of the columns a rank finishes
+        // and of the tokens, and the ranks' receive-area addresses
+        q.smem_bytes = 1024 + (size_t)stages * stage + (size_t)(2 * stages + 4) * 8 + 16 + (256 + 64 + 8) * 4;
+        // No more CTAs of this kernel may share an SM than its tensor memory holds: a CTA
+        // waiting for columns another CTA of the same grid holds, while that one waits for
+        // its cluster peers, would stall the grid.  Shared memory (228 KB per SM, 1 KB
+        // reserved per CTA) bounds the CTAs per SM, so pad the request until it does.
+        {
+            const size_t cols = bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
+            const size_t max_ctas = 512 / cols;
+            while (233472 / (q.smem_bytes + 1024) > max_ctas) q.smem_bytes += 1024;
+        }
+        if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
+        // the partial sums of the columns a rank finishes sit over its stage memory: over the
+        // R stages, for each of the two K-block counts a rank can hold, whose last use comes
+        // earliest (stage s last holds K block s + S floor((n - 1 - s) / S) of n)
+        const size_t recv = (size_t)C * M * (q.sw + 4) * 4;
+        if (recv > (size_t)stages * stage) return W8_ERR_UNSUPPORTED;
+        q.recv_R = (int)((recv + stage - 1) / stage);
+        q.nkb_lo = q.kbs / C;
+        for (int h = 0; h < 2; ++h) {
+            const int n = q.nkb_lo + h;
+            int best = 0x7FFFFFFF;
+            q.recv_first[h] = 0;
+            for (int c0 = 0; c0 + q.recv_R <= stages; ++c0) {
+                int worst = -1;
+                for (int st = c0; st < c0 + q.recv_R; ++st)
+                    worst = std::max(worst, st < n ? st + stages * ((n - 1 - st) / stages) : -1);
+                if (worst < best) { best = worst; q.recv_first[h] = c0; }
+            }
+        }
+        q.nsb = q.kbs;
+        q.rows_R = M;
+        q.rows_C = N;
+        q.r_tiles = 1;
+        q.c_tiles = (N + bn - 1) / bn;
+        q.tiles = q.c_tiles;
+        q.units = (long long)q.tiles * q.kbs;
+        const long long g = (long long)q.tiles * C;
+        if (g > 0x7FFFFFFF) return W8_ERR_UNSUPPORTED;
+        q.G = (int)g;
+        q.align_tiles = 1;
+        q.ws_counters = 0;
+        q.ws_bytes = 0;
+        *p = q;
+        return W8_OK;
+    }
     if (variant & W8_V_PAIR) {
         // 256 x 256 tiles on CTA pairs: Standard full-K loop, FP8-dynamic / INT8
         if (block || q.swap || q.stream || lg != 0 || q.cluster || q.bm != 128 || q.pfix || tid != kTileBN256 ||
@@ -220,6 +292,40 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
 {
     if (p.ws_bytes > 0 && (workspace == nullptr || ws_bytes < p.ws_bytes)) return W8_ERR_WORKSPACE;
     if (p.ws_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return W8_ERR_ALIGNMENT;
+    if (p.decode) {
+        // token box of M rounded up to 8 rows, weight box of bn rows
+        GemmMaps maps;
+        if (!make_tmap(&maps.R, A_q, p.M, p.K, p.m8)) return W8_ERR_CUDA;
+        if (!make_tmap(&maps.C, W_q, p.N, p.K, p.bn)) return W8_ERR_CUDA;
+        GemmArgs args = {};
+        args.M = p.M; args.N = p.N; args.K = p.K;
+        args.rows_R = p.M; args.rows_C = p.N;
+        args.r_tiles = 1; args.c_tiles = p.c_tiles; args.tiles = p.tiles;
+        args.kbs = p.kbs;
+        args.nsb = p.kbs;
+        args.units = p.units;
+        args.G = p.G;
+        args.align_tiles = 1;
+        args.csplit = p.split;
+        args.stages = p.stages;
+        args.pdl = p.pdl;
+        args.vec_ok = (p.N % 8 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
+        args.sA = A_scale;
+        args.sW = W_scale;
+        args.out = static_cast<__nv_bfloat16*>(out);
+        args.out_i32 = out_i32;
+        args.bn = p.bn;
+        args.m8 = p.m8;
+        args.l2ahead = p.l2ahead;
+        args.sw = p.sw;
+        args.recv_R = p.recv_R;
+        args.nkb_lo = p.nkb_lo;
+        args.recv_first[0] = p.recv_first[0];
+        args.recv_first[1] = p.recv_first[1];
+        const cudaError_t e = launch_decode(p, maps, args, s);
+        if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
+        return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
+    }
     CUtensorMap tR, tC;
     const void* R = p.swap ? W_q : A_q;
     const void* C = p.swap ? A_q : W_q;
@@ -399,7 +505,8 @@ int gemm_occupancy(const GemmPlan& p, int* n)
     maps.occupancy = n;
     GemmArgs args = {};
     cudaError_t e = cudaErrorInvalidValue;
-    if (p.fq)                      e = launch_fq(p, maps, args, nullptr);
+    if (p.decode)                  e = launch_decode(p, maps, args, nullptr);
+    else if (p.fq)                 e = launch_fq(p, maps, args, nullptr);
     else if (p.grouped)            e = launch_grouped(p, maps, args, nullptr);
     else if (p.pair)               e = launch_pair(p, maps, args, nullptr);
     else if (p.fmt >= W8_FMT_BLOCK_FP8) e = launch_block(p, maps, args, nullptr);
@@ -414,7 +521,8 @@ int gemm_occupancy(const GemmPlan& p, int* n)
 int gemm_device_status(int clear)
 {
     int first = 0;
-    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq, status_grouped, status_pair}) {
+    for (int (*f)(int) : {status_f8, status_i8, status_block, status_bm64, status_fq, status_grouped, status_pair,
+                          status_decode}) {
         const int v = f(clear);
         if (v == W8_ERR_CUDA) return v;
         if (v != 0 && first == 0) first = v;

@@ -100,6 +100,14 @@ struct GemmArgs {
     const int* g_off;     // device [g_E + 1]
     uint8_t* dbg_q;       // optional: codes of the K blocks of weight tile 0, [M, K]
     float* dbg_s;         // optional: scales, [M] or [M, K/128]
+    // decode form (w8_gemm_decode.cu)
+    int bn;               // weight rows per tile (64..256, a multiple of 16)
+    int m8;               // token rows of the activation box
+    int l2ahead;          // K blocks of weights prefetched into L2 ahead of the stages
+    int sw;               // columns of the tile each cluster rank finishes
+    int recv_R;           // stages spanned by a rank's receive area
+    int nkb_lo;           // the smaller of the two K-block counts a rank holds
+    int recv_first[2];    // first stage of the receive area for nkb_lo and nkb_lo + 1 K blocks
 };
 
 // K blocks a CTA with units [u0, u1) multiplies: its own range when the units lie in one
@@ -1257,6 +1265,7 @@ cudaError_t launch_bm64(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a,
 cudaError_t launch_fq(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_grouped(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_pair(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s);
 int status_f8(int clear);
 int status_i8(int clear);
 int status_block(int clear);
@@ -1264,6 +1273,7 @@ int status_bm64(int clear);
 int status_fq(int clear);
 int status_grouped(int clear);
 int status_pair(int clear);
+int status_decode(int clear);
 
 }  // namespace gemm
 }  // namespace w8

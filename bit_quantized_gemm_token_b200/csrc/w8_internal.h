@@ -51,6 +51,13 @@ struct GemmPlan {
     int grouped;      // mixture-of-experts form: M = all tokens, N per expert
     int g_E;          // grouped: experts
     int pair;         // 256 x 256 tiles on CTA pairs (cta_group::2 MMA), Standard form
+    int decode;       // decode form: tokens in the 64-row MMA operand, bn weight rows, split = cluster size
+    int m8;           // decode: token rows of the activation box (M rounded up to 8)
+    int l2ahead;      // decode: K blocks of weights kept in flight into L2 ahead of the stages
+    int sw;           // decode: columns of the tile each cluster rank finishes (multiple of 16)
+    int recv_R;       // decode: stages spanned by a rank's receive area
+    int nkb_lo;       // decode: the smaller of the two K-block counts a rank holds
+    int recv_first[2];   // decode: first stage of the receive area for nkb_lo and nkb_lo + 1 K blocks
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile

@@ -42,6 +42,8 @@ W8_V_BM64 = 1 << 18
 W8_V_PFIX = 1 << 19
 W8_V_FUSED = 1 << 24
 W8_V_PAIR = 1 << 25
+W8_V_DECODE = 1 << 26
+W8_V_L2_SHIFT = 27
 W8_V_KPS_SHIFT = 20
 W8_V_CPS_SHIFT = 22
 TILE_BN = {16: 0, 32: 1, 64: 2, 128: 3, 256: 4}
@@ -74,7 +76,28 @@ def variant(swap: bool, split: int = 1, bn: int = 16, stream: bool = False, stag
     return v
 
 
+def decode_variant(bn: int = 256, c: int = 1, stages: int = 0, l2ahead: int = 4, pdl: bool = False) -> int:
+    """Explicit W8_V_DECODE variant word: bn weight rows per tile (64..256, a multiple of
+    16), c K chunks per tile run as one cluster (1..8), stages (0 = default), l2ahead K
+    blocks of weights kept in flight into L2 ahead of the stages."""
+    if bn % 16 or not 64 <= bn <= 256:
+        raise ValueError("bn must be a multiple of 16 in [64, 256]")
+    if not 1 <= c <= 8:
+        raise ValueError("c must be in [1, 8]")
+    if not 0 <= l2ahead <= 15 or not 0 <= stages <= 15:
+        raise ValueError("l2ahead and stages must be in [0, 15]")
+    v = W8_V_EXPLICIT | W8_V_DECODE | ((c - 1) << W8_V_SPLIT_SHIFT) | ((bn // 16 - 1) << W8_V_TILE_SHIFT)
+    v |= (stages << W8_V_STAGES_SHIFT) | (l2ahead << W8_V_L2_SHIFT)
+    if pdl:
+        v |= W8_V_PDL
+    return v
+
+
 def describe(v: int) -> dict:
+    if v & W8_V_DECODE:
+        return {"decode": True, "bn": 16 * (((v >> W8_V_TILE_SHIFT) & 0xF) + 1),
+                "c": ((v >> W8_V_SPLIT_SHIFT) & 0xF) + 1, "stages": (v >> W8_V_STAGES_SHIFT) & 0xF,
+                "l2ahead": (v >> W8_V_L2_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL)}
     inv = {b: k for k, b in TILE_BN.items()}
     return {"swap_ab": bool(v & W8_V_SWAP_AB), "stream": bool(v & W8_V_STREAM),
             "split_k": 1 << ((v >> W8_V_SPLIT_SHIFT) & 0xF), "bn": inv.get((v >> W8_V_TILE_SHIFT) & 0xF),

@@ -52,3 +52,23 @@ def test_variant_round_trip(kw):
 def test_variant_rejects_non_power_of_two_split():
     with pytest.raises(ValueError):
         w8.variant(True, 3, 16)
+
+
+@pytest.mark.parametrize("kw", [dict(bn=256, c=8), dict(bn=176, c=3, stages=2, l2ahead=6, pdl=True), dict(bn=64, c=1)])
+def test_decode_variant_round_trip(kw):
+    v = w8.decode_variant(**kw)
+    d = w8.describe(v)
+    assert d["decode"] and d["bn"] == kw["bn"] and d["c"] == kw["c"]
+    assert d["stages"] == kw.get("stages", 0) and d["l2ahead"] == kw.get("l2ahead", 4) and d["pdl"] == kw.get("pdl", False)
+
+
+def test_decode_variant_legality_without_a_device():
+    # planning needs no GPU: more than 64 tokens, more chunks than K blocks and the
+    # block formats are refused; a legal word resolves to itself
+    v = w8.decode_variant(256, 8)
+    assert w8.w8_gemm_resolve_variant(0, 16, 4096, 4096, v) == v
+    for fmt, M, N, K in [(0, 65, 1024, 1024), (1, 8, 1024, 256), (2, 8, 1024, 1024)]:
+        with pytest.raises(w8.W8Error):
+            w8.w8_gemm_resolve_variant(fmt, M, N, K, w8.decode_variant(256, 3 if K == 256 else 1))
+    with pytest.raises(ValueError):
+        w8.decode_variant(200, 1)
