@@ -1,6 +1,7 @@
 // w8_api.cu -- the C ABI (include/w8.h): argument validation, device check, variant
 // resolution (per-shape table, then a built-in rule) and dispatch to the kernels.
 // Nothing here allocates device memory or synchronises.
+#include <algorithm>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -63,9 +64,9 @@ int table_lookup(int fmt, int N, int K, int M)
 
 namespace {
 
-// Built-in rule when the table has no entry: Swap-AB with the narrowest token tile and the
-// balanced partition for decode-sized M (weights streamed evenly by every SM; the
-// partial-sum traffic stays in L2); the Standard form with whole tiles for prefill.
+// Built-in rule when the table has no entry: the decode form for FP8 / INT8 up to 64
+// tokens; Swap-AB with the narrowest token tile and the balanced partition for Block-FP8
+// decode sizes; CTA-pair (FP8 / INT8) or Standard (Block-FP8) whole tiles for prefill.
 // Grouped GEMM default: Swap-AB over the balanced partition with the narrowest token tile
 // that holds an expert's largest token count (64 beyond that: several token tiles).
 int grouped_variant(int max_m)
@@ -74,9 +75,48 @@ int grouped_variant(int max_m)
     return W8_VARIANT(1, 0, tile, 1);
 }
 
-int builtin_variant(int fmt, int M)
+// Decode form for FP8-dynamic / INT8 at M <= 64: the (weight tile, K chunks) pair with
+// the lowest estimated time on `sms` SMs.  The estimate (microseconds) is the slowest of
+// the HBM stream (~6.5 TB/s), one CTA's stream (~54 GB/s: ~108 KB in flight per SM over
+// ~2 us of latency under load) and its chain of tensor-core instructions (~0.084 us per
+// 64 x BN x 32 MMA), plus ~0.25 us per K chunk for the exchange in distributed shared
+// memory -- the costs measured on B200 for the decode shapes.  0 when none is legal.
+int decode_builtin(int fmt, int M, int N, int K, int sms)
+{
+    const int kbs = (K + 127) / 128;
+    double best_t = 1e30;
+    int best = 0, best_g = 0;
+    for (int bn = 256; bn >= 64; bn -= 16) {
+        const int tiles = (N + bn - 1) / bn;
+        for (int c = 1; c <= 8 && c <= kbs; ++c) {
+            const int g = tiles * c;
+            if (g > sms) break;
+            const int kb = (kbs + c - 1) / c;
+            const double t_hbm = (double)N * K / 6.5e6;
+            const double t_cta = (double)bn * kb * 128 / 54e3;
+            const double t_mma = kb * 4 * 0.084;
+            const double t = std::max(t_hbm, std::max(t_cta, t_mma)) + (c > 1 ? 0.25 * c : 0.0);
+            // ties: the launch with more CTAs (more requests in flight)
+            if (t < best_t - 1e-9 || (t < best_t + 1e-9 && g > best_g)) {
+                const int v = W8_V_EXPLICIT | W8_V_DECODE | ((c - 1) << W8_V_SPLIT_SHIFT) | ((bn / 16 - 1) << W8_V_TILE_SHIFT);
+                GemmPlan plan;
+                if (gemm_plan(fmt, M, N, K, v, sms, &plan) != W8_OK) continue;
+                best_t = t;
+                best = v;
+                best_g = g;
+            }
+        }
+    }
+    return best;
+}
+
+int builtin_variant(int fmt, int M, int N, int K, int sms)
 {
     const bool block = fmt >= W8_FMT_BLOCK_FP8;
+    if (!block && M <= 64) {
+        const int v = decode_builtin(fmt, M, N, K, sms);
+        if (v) return v;
+    }
     if (M <= 16) return W8_VARIANT(1, 0, kTileBN16, 1);
     if (M <= 32) return W8_VARIANT(1, 0, kTileBN32, 1);
     if (M <= 64) return W8_VARIANT(1, 0, kTileBN64, 1);
@@ -96,7 +136,7 @@ int resolve(int fmt, int M, int N, int K, int variant, int sms, GemmPlan* plan)
     if (!(v & W8_V_EXPLICIT)) {
         const int pdl = v & W8_V_PDL;   // AUTO may still ask for PDL
         v = table_lookup(fmt, N, K, M);
-        if (!v) v = builtin_variant(fmt, M);
+        if (!v) v = builtin_variant(fmt, M, N, K, sms);
         v |= pdl;
     }
     const int rc = gemm_plan(fmt, M, N, K, v, sms, plan);

@@ -16,7 +16,8 @@ it in the layer's order (qkv -> o -> gate_up -> down -> qkv), and the candidate 
 lowest time for the two pairs wins.  A first pass puts the built-in choice in front; a
 second pass re-times the best few behind the first pass's winners.
 
-    python -m bit_quantized_gemm_token_b200.sweep [--out PATH] [--quick] [--resume]
+    python -m bit_quantized_gemm_token_b200.sweep [--out PATH] [--quick] [--formats 0,1,2]
+                                                  [--families swap,bm64,decode,shipped]
 """
 import argparse
 import json
@@ -34,9 +35,65 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 DEFAULT_OUT = os.path.join(HERE, "tuning", "b200_table.txt")
 
 
-def candidates(fmt, M, N, K, quick=False):
+def decode_estimate(M, N, K, bn, c):
+    """Microseconds the built-in rule estimates for the decode form (the same model as
+    the library's: HBM stream, one CTA's stream, its MMA chain, the cluster exchange)."""
+    kbs = -(-K // 128)
+    kb = -(-kbs // c)
+    t = max(N * K / 6.5e6, bn * kb * 128 / 54e3, kb * 4 * 0.084)
+    return t + (0.25 * c if c > 1 else 0.0)
+
+
+def decode_candidates(fmt, M, N, K, sms=148, keep=10):
+    """Decode-form variants (FP8 / INT8, M <= 64): the `keep` (tile, K chunks) pairs the
+    model ranks best among those filling 60-100% of the SMs, each at the default pipeline
+    depth and at a deeper one."""
+    if fmt >= 2 or M > 64:
+        return []
+    kbs = -(-K // 128)
+    pairs = []
+    for bn in range(64, 257, 16):
+        tiles = -(-N // bn)
+        for c in range(1, 9):
+            if c > kbs or tiles * c > sms or tiles * c < 0.6 * sms:
+                continue
+            pairs.append((decode_estimate(M, N, K, bn, c), bn, c))
+    pairs.sort()
+    out = []
+    m8 = (M + 7) // 8 * 8
+    for _, bn, c in pairs[:keep]:
+        stage = (m8 + bn) * 128
+        deep = min(8, 196608 // stage)
+        for st in sorted({0, deep}):
+            out.append(w8.decode_variant(bn, c, stages=st, l2ahead=0))
+    return out
+
+
+def shipped_variant(fmt, M, N, K):
+    """The variant the table shipped with the package resolves to (0 if none)."""
+    best = None
+    if os.path.exists(DEFAULT_OUT):
+        for line in open(DEFAULT_OUT):
+            f = line.split("#")[0].split()
+            if len(f) != 5:
+                continue
+            r = [int(x) for x in f[:4]] + [int(f[4], 16)]
+            if r[0] == fmt and r[1] == N and r[2] == K and r[3] >= M and (best is None or r[3] < best[3]):
+                best = r
+    return best[4] if best else 0
+
+
+def candidates(fmt, M, N, K, quick=False, families=("swap", "bm64", "decode")):
     block = fmt >= 2
     out = []
+    if "decode" in families:
+        out += decode_candidates(fmt, M, N, K)
+    if "shipped" in families:
+        v = shipped_variant(fmt, M, N, K)
+        if v:
+            out.append(v)
+    if "swap" not in families:
+        return _legal(fmt, M, N, K, out)
     bns = [b for b in (16, 32, 64) if b >= min(M, 64)][:2]
     for bn in bns:
         parts = [("stream", 1), ("stream", 2)] + [("split", s) for s in (1, 2, 4, 8, 16)] + \
@@ -49,7 +106,7 @@ def candidates(fmt, M, N, K, quick=False):
                     else:
                         v = w8.variant(True, arg, bn, stages=stages, kps=kps, cluster=(kind == "cluster"))
                     out.append(v)
-    if not block:
+    if not block and "bm64" in families:
         # Standard form, 64-row token tile, weights in the MMA's N slot
         for bn in (128, 256):
             parts = [("stream", 1), ("split", 1), ("split", 2), ("split", 4), ("split", 8), ("cluster", 2), ("cluster", 4),
@@ -73,6 +130,10 @@ def candidates(fmt, M, N, K, quick=False):
                         else:
                             v = w8.variant(False, arg, bn, stages=stages, kps=kps, bm64=True, pfix=True)
                         out.append(v)
+    return _legal(fmt, M, N, K, out)
+
+
+def _legal(fmt, M, N, K, out):
     legal = []
     for v in out:
         try:
@@ -181,6 +242,7 @@ def time_in_context(prev, pv, prob, M, v, reps=2):
 
 
 def default_variant(fmt, M):
+    """The reference every candidate's output is checked against: Swap-AB, balanced."""
     bn = 16 if M <= 16 else 32 if M <= 32 else 64
     return w8.variant(True, 1, bn, stream=True)
 
@@ -190,8 +252,22 @@ def main():
     ap.add_argument("--out", default=DEFAULT_OUT)
     ap.add_argument("--quick", action="store_true", help="default pipeline depths only")
     ap.add_argument("--formats", default="0,1,2")
+    ap.add_argument("--families", default="swap,bm64,decode",
+                    help="candidate families: swap (Swap-AB), bm64 (64-row token tile), decode, shipped (the "
+                         "current table's entry)")
     ap.add_argument("--log", default="")
     args = ap.parse_args()
+    families = tuple(args.families.split(","))
+    # rows of formats not swept now are kept from the table being replaced
+    kept = []
+    fmts_swept = set()
+    for f in args.formats.split(","):
+        fmts_swept |= {2, 3} if int(f) == 2 else {int(f)}
+    if os.path.exists(args.out):
+        for line in open(args.out):
+            f = line.split("#")[0].split()
+            if len(f) == 5 and int(f[0]) not in fmts_swept:
+                kept.append((int(f[0]), int(f[1]), int(f[2]), int(f[3]), int(f[4], 16)))
     os.environ["W8_TABLE"] = "none"
     w8.w8_clear_table()
     dev = torch.device("cuda", 0)
@@ -209,7 +285,7 @@ def main():
             cands = []
             for prob in probs:
                 ok = []
-                for v in candidates(fmt, M, prob.N, prob.K, args.quick):
+                for v in candidates(fmt, M, prob.N, prob.K, args.quick, families):
                     if prob.check(M, v, ref_v):
                         ok.append(v)
                     else:
@@ -243,6 +319,7 @@ def main():
                     rows.append((f, N, K, M, best_v))
         del probs
         torch.cuda.empty_cache()
+    rows += kept
     rows.sort(key=lambda r: (r[0], r[2], r[1], r[3]))
     os.makedirs(os.path.dirname(args.out), exist_ok=True)
     with open(args.out, "w") as fh:

@@ -97,9 +97,10 @@ def describe(v: int) -> dict:
     if v & W8_V_DECODE:
         return {"decode": True, "bn": 16 * (((v >> W8_V_TILE_SHIFT) & 0xF) + 1),
                 "c": ((v >> W8_V_SPLIT_SHIFT) & 0xF) + 1, "stages": (v >> W8_V_STAGES_SHIFT) & 0xF,
-                "l2ahead": (v >> W8_V_L2_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL)}
+                "l2ahead": (v >> W8_V_L2_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL),
+                "swap_ab": False, "stream": False, "cluster": False, "bm64": False, "pfix": False, "pair": False}
     inv = {b: k for k, b in TILE_BN.items()}
-    return {"swap_ab": bool(v & W8_V_SWAP_AB), "stream": bool(v & W8_V_STREAM),
+    return {"decode": False, "swap_ab": bool(v & W8_V_SWAP_AB), "stream": bool(v & W8_V_STREAM),
             "split_k": 1 << ((v >> W8_V_SPLIT_SHIFT) & 0xF), "bn": inv.get((v >> W8_V_TILE_SHIFT) & 0xF),
             "stages": (v >> W8_V_STAGES_SHIFT) & 0xF, "pdl": bool(v & W8_V_PDL),
             "kps": (v >> W8_V_KPS_SHIFT) & 0x3, "cps": (v >> W8_V_CPS_SHIFT) & 0x3,

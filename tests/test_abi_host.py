@@ -105,11 +105,16 @@ def test_linear_and_grouped_planning(L):
 
 def test_variant_resolution_and_workspace(L):
     w8.w8_clear_table()   # the built-in rule, not the shipped table
-    # decode: Swap-AB with the narrow token tile, balanced partition
-    v = w8.w8_gemm_resolve_variant(0, 1, 4096, 4096)
-    d = w8.describe(v)
+    # decode sizes, FP8 / INT8: the decode form on at most one wave of CTAs
+    for fmt in (0, 1):
+        for M in (1, 32, 64):
+            d = w8.describe(w8.w8_gemm_resolve_variant(fmt, M, 4096, 4096))
+            assert d["decode"] and 64 <= d["bn"] <= 256 and 1 <= d["c"] <= 8
+            assert -(-4096 // d["bn"]) * d["c"] <= 148
+    # Block-FP8 decode: Swap-AB with the narrow token tile, balanced partition
+    d = w8.describe(w8.w8_gemm_resolve_variant(2, 1, 4096, 4096))
     assert d["swap_ab"] and d["stream"] and d["bn"] == 16
-    assert w8.describe(w8.w8_gemm_resolve_variant(0, 32, 4096, 4096))["bn"] == 32
+    assert w8.describe(w8.w8_gemm_resolve_variant(2, 32, 4096, 4096))["bn"] == 32
     assert not w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["swap_ab"]
     # past 64 tokens: CTA pairs (FP8 / INT8); Block-FP8 keeps its tile
     assert w8.describe(w8.w8_gemm_resolve_variant(0, 4096, 4096, 4096))["pair"]
@@ -147,7 +152,8 @@ def test_variant_resolution_and_workspace(L):
     n = w8.w8_gemm_workspace_size(0, 8, 256, 1024, w8.variant(True, split=4, bn=16))
     ctas = 2 * 4                                  # 2 tiles x split 4
     assert n == 65536 * 4 + ctas * 2 * 16 * 128 * 4
-    assert w8.w8_gemm_workspace_size(0, 8, 4096, 4096, 0) > 0
+    assert w8.w8_gemm_workspace_size(2, 8, 4096, 4096, 0) > 0     # Block-FP8 decode: balanced partition
+    assert w8.w8_gemm_workspace_size(0, 8, 4096, 4096, 0) == 0    # decode form: reduced in the cluster
 
 
 def test_table_parsing(L, tmp_path):
@@ -159,7 +165,7 @@ def test_table_parsing(L, tmp_path):
         assert w8.w8_load_table(str(p)) == 2
         assert w8.w8_gemm_resolve_variant(0, 8, 4096, 4096) == v1
         assert w8.w8_gemm_resolve_variant(0, 17, 4096, 4096) == v2
-        assert w8.describe(w8.w8_gemm_resolve_variant(0, 8, 4096, 6144))["stream"]   # not in table
+        assert w8.describe(w8.w8_gemm_resolve_variant(0, 8, 4096, 6144))["decode"]   # not in table: built-in rule
         bad = tmp_path / "bad.txt"
         bad.write_text("0 4096 4096 16\n")
         assert L.w8_load_table(os.fsencode(str(bad))) == w8.W8_ERR_IO
