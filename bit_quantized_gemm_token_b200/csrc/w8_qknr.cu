@@ -4,7 +4,7 @@
 //
 // For qkv[T, (Hq + 2 Hkv) * D] bf16 (query heads, key heads, value heads; D values each)
 // and every token t and query or key head:
-//   y_k = (x_k * r) * w_k,  r = 1 / sqrt(ss / D + eps),  ss = sum x_k^2 (fp64, then fp32),
+//   y_k = (x_k * r) * w_k,  r = 1 / sqrt(ss / D + eps),  ss = sum x_k^2 (exact, then fp32),
 //   w = the query or key head-dimension weight;
 //   with c_i, s_i the cosine / sine row of the token's position (table input,
 //   fp32 [max_pos, D]: cosines then sines), each pair (y_i, y_{i+D/2}) is rotated:
@@ -19,6 +19,7 @@
 
 #include "w8_internal.h"
 #include "w8_ptx.cuh"
+#include "w8_sumsq.cuh"
 
 namespace w8 {
 namespace {
@@ -91,16 +92,16 @@ __global__ void __launch_bounds__(128) qk_norm_rope_kernel(const __nv_bfloat16* 
         float lo[C], hi[C];
         unpack(lov[j], lo);
         unpack(hiv[j], hi);
-        // sum of squares: each square of a bf16 is exact in fp64; lane sums, then a fixed tree
-        double ss = 0.0;
+        // the exact sum of squares rounded once to fp32 (w8_sumsq.cuh): lane sums, then the warp
+        DSum ss{0.0, 0.0};
 #pragma unroll
         for (int i = 0; i < C; ++i) {
-            ss = __fma_rn((double)lo[i], (double)lo[i], ss);
-            ss = __fma_rn((double)hi[i], (double)hi[i], ss);
+            ss = dsum_sq(ss, lo[i]);
+            ss = dsum_sq(ss, hi[i]);
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
-        const float mean = __fdiv_rn(__double2float_rn(ss), (float)D);
+        for (int off = 16; off > 0; off >>= 1) ss = dsum_add(ss, dsum_shfl_xor(ss, off));
+        const float mean = __fdiv_rn(dsum_to_f32(ss), (float)D);
         const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
         const __nv_bfloat16* w = (h < Hq) ? qw : kw;
         float wl[C], wh[C];

@@ -24,6 +24,7 @@
 #include "w8_codes.cuh"
 #include "w8_internal.h"
 #include "w8_ptx.cuh"
+#include "w8_sumsq.cuh"
 
 namespace w8 {
 namespace {
@@ -48,17 +49,17 @@ __device__ __forceinline__ float block_max(float v, float* red)
     return r;
 }
 
-// Sum over the CTA in fp64 with a fixed reduction tree; every thread gets the result.
-__device__ __forceinline__ double block_sum_f64(double v, double* red)
+// Double-double sum over the CTA; every thread gets the result.  `red` holds 32 DSums.
+__device__ __forceinline__ DSum block_sum_dd(DSum v, DSum* red)
 {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    for (int o = 16; o > 0; o >>= 1) v = dsum_add(v, dsum_shfl_xor(v, o));
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     if (l == 0) red[w] = v;
     __syncthreads();
-    double r = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0;
+    DSum r = (l < (int)(blockDim.x >> 5)) ? red[l] : DSum{0.0, 0.0};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xFFFFFFFFu, r, o);
+    for (int o = 16; o > 0; o >>= 1) r = dsum_add(r, dsum_shfl_xor(r, o));
     __syncthreads();
     return r;
 }
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
                                                              int H, int ldx, uint8_t* __restrict__ q,
                                                              float* __restrict__ scale, int ue8m0)
 {
-    __shared__ double redd[32];
+    __shared__ DSum redd[32];
     __shared__ float red[32];
     ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
     const int chunks = H >> 3;
     const __nv_bfloat16* xr = x + (size_t)m * ldx;
     uint4 raw[CPT];
-    double ss = 0.0;
+    DSum ss{0.0, 0.0};
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
         const int idx = threadIdx.x + c * blockDim.x;
@@ -239,14 +240,12 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
             float f[8];
             unpack_bf16x8(raw[c], f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const double d = (double)f[i];
-                ss = __fma_rn(d, d, ss);   // the square of a bf16 value is exact in fp64
-            }
+            for (int i = 0; i < 8; ++i) ss = dsum_sq(ss, f[i]);
         }
     }
-    ss = block_sum_f64(ss, redd);
-    const float mean = __fdiv_rn(__double2float_rn(ss), (float)H);
+    ss = block_sum_dd(ss, redd);
+    // the exact sum of squares rounded once to fp32, then the mean (w8_sumsq.cuh)
+    const float mean = __fdiv_rn(dsum_to_f32(ss), (float)H);
     const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
     if (GROUPED) {
         // rms_norm_per_block_quant: y = (x * r) * gamma, then one scale per 1x128 group

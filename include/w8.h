@@ -192,7 +192,8 @@ W8_API int w8_quant_weight_block(const void* w, int N, int K, void* q, float* sc
 /* Fused rms_norm + dynamic per-token fp8 quant, one launch ([FP8] "Patron de fusion
  * del forward pass": rms_norm + fp8_quant; "Kernels Helion implementados":
  * rms_norm_dynamic_per_token_quant).  Per row:
- *   ss = sum x^2 accumulated in fp64, rounded to fp32; r = 1/sqrt(ss/H + eps) (fp32,
+ *   ss = sum x^2, the exact sum rounded once to fp32 (nearest, ties to even; any
+ *   summation order gives it); r = 1/sqrt(ss/H + eps) (fp32,
  *   correctly rounded steps); y = (x * r) * gamma in fp32 (never rounded to bf16);
  *   then the per-token fp8 quantization of y.
  *   x bf16 [M, H] (row stride ldx), gamma bf16 [H]; q e4m3 [M, H]; scale fp32 [M].
@@ -293,7 +294,7 @@ W8_API size_t w8_grouped_gemm_workspace_size(int fmt, int E, int T, int N, int K
  *   qkv, out  bf16 [T, (Hq + 2*Hkv) * D] row-major: Hq query heads, Hkv key heads, Hkv
  *             value heads, D contiguous values each; out may equal qkv (in place);
  *   for each token t and query (key) head: y = rms_norm(head) with q_weight (k_weight)
- *             [D] bf16 -- sum of squares in fp64 rounded once to fp32, r = 1/sqrt(ss/D
+ *             [D] bf16 -- the exact sum of squares rounded once to fp32, r = 1/sqrt(ss/D
  *             + eps), y_k = (x_k * r) * w_k in fp32 -- then each pair (y_i, y_{i+D/2}) is
  *             rotated by the angle of position p = positions[t]: o_i = y_i c_i -
  *             y_{i+D/2} s_i, o_{i+D/2} = y_{i+D/2} c_i + y_i s_i, c_i = cos_sin[p*D + i],

@@ -114,3 +114,36 @@ def test_silu_mul_quant_group_bit_exact(orc, M, I, ue8m0):
     oq, os_ = orc.silu_mul_quant_group(bits(xgu), 128, ue8m0)
     assert np.array_equal(s.cpu().numpy(), os_)
     assert np.array_equal(u8(q), oq)
+
+
+def _midpoint_rows(H):
+    """Rows whose exact sum of squares lies on, or a hair past, an fp32 rounding midpoint
+    (1 + 2^-24 between 1 and the next fp32 value): a running fp64 sum rounds the second
+    and third the wrong way."""
+    rows = np.zeros((3, H), dtype=np.float32)
+    rows[0, :2] = [1.0, 2.0 ** -12]                       # on the midpoint: ties to even (1)
+    rows[1, :3] = [1.0, 2.0 ** -12, 2.0 ** -50]           # just past it: rounds up
+    rows[2, 0] = 1.0                                      # 4096 squares of 2^-36 add to 2^-24, one more past it
+    rows[2, 1:4097] = 2.0 ** -18
+    rows[2, H - 1] = 2.0 ** -60
+    return torch.from_numpy(rows).to(torch.bfloat16)
+
+
+def test_rmsnorm_sum_of_squares_at_fp32_midpoints(orc):
+    """The sum of squares is the exact sum rounded once to fp32, whatever the order the
+    GPU adds in: with gamma = 1 and eps = 0 the scale is RN(RN(1 * r) / 448) with r =
+    1 / sqrt(ss / H), which moves with the last bit of ss."""
+    H = 8192
+    x = _midpoint_rows(H)
+    g = torch.ones(H, dtype=torch.bfloat16)
+    q, s = w8.w8_rmsnorm_quant(x.cuda(), g.cuda(), 0.0)
+    oq, os_ = orc.rmsnorm_quant(bits(x), bits(g), 0.0)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
+    # the rows do test the rounding: an fp64 running sum would give other scales for
+    # the rows past the midpoint
+    xf = x.float().numpy().astype(np.float64)
+    for i in (1, 2):
+        naive = np.float32(np.sum(xf[i] * xf[i]))
+        r = np.float32(1.0) / np.sqrt(naive / np.float32(H))
+        assert np.float32(r / np.float32(448.0)) != os_[i]
