@@ -243,6 +243,38 @@ def gemm(fmt, Aq, sA, Wq, sW, n_lo=0, n_hi=None):
     return out, ref, acc
 
 
+def gemm_ref_matmul(fmt, Aq, sA, Wq, sW):
+    """The fp64 reference of orc_gemm (ref_f64) for every output, with numpy's matmul as
+    the summation step: the codes are decoded with the oracle's own decoder (int8, or
+    orc_e4m3_decode through a 256-entry table), each sum of products is exact in fp64 at
+    these sizes (products of 8-bit values span < 2^36 and at most 2^15 of them are added),
+    so any summation order gives orc_gemm's value; the scales are applied in orc_gemm's
+    order -- (acc * sA) * sW, or per K block (sA * sW) * part added in block order.  For
+    checking full-size outputs, where the C loop would take minutes."""
+    Aq, sA, Wq, sW = _gemm_args(Aq, sA, Wq, sW)
+    M, K = Aq.shape
+    if fmt == FMT_INT8:
+        a = Aq.view(np.int8).astype(np.float64)
+        w = Wq.view(np.int8).astype(np.float64)
+    else:
+        table = e4m3_decode(np.arange(256, dtype=np.uint8))
+        a = table[Aq]
+        w = table[Wq]
+    if fmt != FMT_BLOCK_FP8:
+        acc = a @ w.T
+        return (acc * sA.astype(np.float64)[:, None]) * sW.astype(np.float64)[None, :]
+    nbk = (K + 127) // 128
+    N = Wq.shape[0]
+    ref = np.zeros((M, N), dtype=np.float64)
+    sW2 = sW.reshape(-1, nbk).astype(np.float64)
+    sA2 = sA.reshape(M, nbk).astype(np.float64)
+    for kb in range(nbk):
+        part = a[:, kb * 128:(kb + 1) * 128] @ w[:, kb * 128:(kb + 1) * 128].T
+        sc = sA2[:, kb][:, None] * sW2[np.arange(N) // 128, kb][None, :]
+        ref += sc * part
+    return ref
+
+
 def gemm_points(fmt, Aq, sA, Wq, sW, pm, pn):
     Aq, sA, Wq, sW = _gemm_args(Aq, sA, Wq, sW)
     M, K = Aq.shape

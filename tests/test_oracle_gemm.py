@@ -161,3 +161,21 @@ def test_column_slice_matches_full(orc):
     out, ref, _ = orc.gemm(0, Aq, sA, Wq, sW)
     out2, ref2, _ = orc.gemm(0, Aq, sA, Wq, sW, n_lo=100, n_hi=229)
     assert np.array_equal(ref[:, 100:229], ref2) and np.array_equal(out[:, 100:229], out2)
+
+
+@pytest.mark.parametrize("fmt,M,N,K", [(0, 5, 300, 640), (1, 7, 260, 1040), (2, 3, 384, 768), (0, 33, 129, 4096),
+                                       (2, 9, 200, 1280)])
+def test_matmul_reference_equals_the_loop(orc, fmt, M, N, K):
+    """gemm_ref_matmul (numpy's matmul over the oracle's decoded codes, for full-size
+    checks) gives orc_gemm's fp64 reference bit for bit: the sums of products are exact
+    in fp64 at these sizes and the scales are applied in the same order."""
+    x = synth.activations(M, K, seed=600 + fmt)
+    w = synth.weights(N, K, seed=601 + fmt)
+    if fmt == 2:
+        Aq, sA = orc.quant_rows(0, synth.bf16_bits(x), group=128)
+        Wq, sW = orc.quant_weight_block(synth.bf16_bits(w))
+    else:
+        Aq, sA = orc.quant_rows(fmt, synth.bf16_bits(x))
+        Wq, sW = orc.quant_rows(fmt, synth.bf16_bits(w))
+    _, ref, _ = orc.gemm(fmt, Aq, sA, Wq, sW)
+    assert np.array_equal(orc.gemm_ref_matmul(fmt, Aq, sA, Wq, sW), ref)

@@ -139,6 +139,12 @@ PY_MUTANTS = [
     ("grouped GEMM uses the first expert's scales",
      "np.asarray(Wq)[e], np.asarray(sW)[e])",
      "np.asarray(Wq)[e], np.asarray(sW)[0])"),
+    ("matmul reference applies the weight scale per token",
+     "return (acc * sA.astype(np.float64)[:, None]) * sW.astype(np.float64)[None, :]",
+     "return (acc * sA.astype(np.float64)[:, None]) * sW.astype(np.float64)[:acc.shape[0], None]"),
+    ("matmul reference takes the next block's weight scale",
+     "sc = sA2[:, kb][:, None] * sW2[np.arange(N) // 128, kb][None, :]",
+     "sc = sA2[:, kb][:, None] * sW2[np.arange(N) // 128, (kb + 1) % nbk][None, :]"),
     ("grouped GEMM does not slice the token scales",
      "np.asarray(sA)[lo:hi]",
      "np.asarray(sA)[:hi - lo]"),
