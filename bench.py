@@ -64,7 +64,7 @@ def load_peaks():
 
 def gemm_source_hash():
     h = hashlib.sha256()
-    for f in ("w8_gemm_kernel.cuh", "w8_gemm.cu", "w8_ptx.cuh"):
+    for f in ("w8_gemm_kernel.cuh", "w8_gemm.cu", "w8_ptx.cuh", "w8_gemm_decode.cu"):
         with open(os.path.join(ROOT, "bit_quantized_gemm_token_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -369,6 +369,76 @@ def time_graph(fn, steps, warmup, world, clock=None):
     barrier(world)
     del g
     return ms, launches
+
+
+BLOCK_SHAPES = [(5120, 10240), (5120, 51200), (25600, 5120), (4096, 6144)]
+
+
+def short_variant(v):
+    from bit_quantized_gemm_token_b200 import w8
+    d = w8.describe(v)
+    if d["decode"]:
+        return "decode bn%d c%d st%d" % (d["bn"], d["c"], d["stages"])
+    form = "pair" if d["pair"] else "swap" if d["swap_ab"] else "std"
+    part = "stream" if d["stream"] else ("cluster%d" % d["split_k"]) if d["cluster"] else ("split%d" % d["split_k"])
+    return "%s bn%d %s" % (form, d["bn"], part)
+
+
+def time_decode_table(dev, peak, reps=10):
+    """Every (format, shape, M) of the decode workloads timed alone: the GEMM (AUTO +
+    programmatic dependent launch) replayed from a CUDA graph against enough weight copies
+    to exceed 3x the L2, so each launch streams its weights from HBM.  Per entry: K, N, M,
+    microseconds, TB/s of algorithmic bytes and the fraction of the measured copy peak,
+    and the variant AUTO resolved to; per format the weight-byte-weighted aggregate
+    (total bytes / total time)."""
+    import torch
+    from bit_quantized_gemm_token_b200 import w8
+    g = torch.Generator(device=dev)
+    g.manual_seed(777)
+    out = {}
+    for name, fmt, shapes in (("fp8_dynamic", w8.W8_FMT_FP8_DYN, SHAPES), ("w8a8_int8", w8.W8_FMT_INT8, SHAPES),
+                              ("block_fp8", w8.W8_FMT_BLOCK_FP8, BLOCK_SHAPES)):
+        block = fmt >= w8.W8_FMT_BLOCK_FP8
+        rows, tot_b, tot_us = [], 0, 0.0
+        for (K, N) in shapes:
+            ncopy = max(2, -(-400_000_000 // (N * K)))
+            W = []
+            for _ in range(ncopy):
+                wb = (torch.randn(N, K, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+                W.append(w8.w8_quant_weight_block(wb) if block else
+                         w8.w8_quant_per_token(wb, w8.W8_Q_INT8 if fmt == w8.W8_FMT_INT8 else w8.W8_Q_FP8))
+                del wb
+            ws = w8.Workspace(dev)
+            for M in MS:
+                x = torch.randn(M, K, device=dev, generator=g).to(torch.bfloat16)
+                if block:
+                    A, sA = w8.w8_quant_per_token(x, w8.W8_Q_FP8, group=128)
+                else:
+                    A, sA = w8.w8_quant_per_token(x, w8.W8_Q_INT8 if fmt == w8.W8_FMT_INT8 else w8.W8_Q_FP8)
+                o = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+                v = w8.W8_VARIANT_AUTO | w8.W8_V_PDL
+
+                def rot():
+                    for Wq, sW in W:
+                        w8.w8_gemm(fmt, A, sA, Wq, sW, out=o, variant=v, workspace=ws)
+                    return len(W)
+                ms, n = time_graph(rot, reps, 3, 1)
+                us = ms * 1e3 / n
+                if block:
+                    b = N * K + 4 * ((N + 127) // 128) * (K // 128) + M * K + 4 * M * (K // 128) + 2 * M * N
+                else:
+                    b = gemm_bytes(M, N, K)
+                tot_b += b
+                tot_us += us
+                tbs = b / us / 1e6
+                rows.append([K, N, M, round(us, 2), round(tbs, 3), round(tbs * 1e3 / peak, 4),
+                             short_variant(w8.w8_gemm_resolve_variant(fmt, M, N, K))])
+            del W, ws
+            torch.cuda.empty_cache()
+        agg = tot_b / tot_us / 1e6
+        out[name] = {"rows": rows, "weighted_TB/s": round(agg, 3), "weighted_frac": round(agg * 1e3 / peak, 4)}
+    out["columns"] = ["K", "N", "M", "us", "TB/s", "frac of measured copy peak", "variant"]
+    return out
 
 
 def time_extras(dev, peak):
@@ -783,7 +853,7 @@ def run_ours(args):
                      "frac": round(achieved / peak, 4), "peak_source": peak_kind,
                      "traffic": (round(traffic) if traffic is not None else None),
                      "algorithmic_bytes_per_launch": round(gb / n_gemm_per_step),
-                     "kernel": "gemm_kernel (w8_gemm FP8-dynamic)", "ms_gemm_per_step": round(ms_gemm, 4),
+                     "kernel": "gemm_decode_kernel (w8_gemm FP8-dynamic, decode form)", "ms_gemm_per_step": round(ms_gemm, 4),
                      "frac_of_8TBs": round(achieved / 8000.0, 4)},
         "gpu_launches": launches * args.steps,
     }
@@ -797,6 +867,9 @@ def run_ours(args):
     # would sit idle, holding their GPUs, while rank 0 times them)
     if rank == 0 and world == 1 and not args.no_extras:
         out["other_kernels"] = time_extras(dev, peak)
+        out["kernels"] = time_kernels(dev, peak, peak_tflops())
+    if rank == 0 and world == 1 and not args.no_table:
+        out["decode_table"] = time_decode_table(dev, peak)
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(shapes, ms, target_s=args.cpu_seconds)
     if rank == 0:
@@ -836,6 +909,156 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+KERNEL_CASES = ("quant_rows", "quant_rows_int8", "group128", "rmsnorm_quant", "silu_mul_quant", "qk_norm_rope",
+                "gemm_fp8", "gemm_int8", "gemm_block", "grouped", "pair_prefill")
+
+
+def kernel_case(case, dev, g):
+    """One hot-path kernel on a profiling-sized case: (launch function, algorithmic bytes
+    per launch, FLOPs per launch or 0).  The quantizers and producers at 16384 (silu: 4096)
+    rows, query/key norm + rotary embedding at 16384 tokens, the decode GEMMs at M = 8 on
+    4096 x 24576 (Block-FP8: 5120 x 51200), the grouped GEMM at a decode routing, the
+    prefill GEMM at M = 4096.  Bytes count each input once and each output once."""
+    import torch
+    from bit_quantized_gemm_token_b200 import w8
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, device=dev, generator=g) * scale).to(torch.bfloat16)
+    flops = 0
+    if case in ("quant_rows", "quant_rows_int8", "group128"):
+        M, K = 16384, 4096
+        x = rnd(M, K)
+        grp = 128 if case == "group128" else 0
+        qf = w8.W8_Q_INT8 if case == "quant_rows_int8" else w8.W8_Q_FP8
+        q = torch.empty(M, K, dtype=torch.int8 if qf == w8.W8_Q_INT8 else torch.float8_e4m3fn, device=dev)
+        s = torch.empty(M, K // 128, device=dev) if grp else torch.empty(M, device=dev)
+        f = lambda: w8.w8_quant_per_token(x, qf, group=grp, q=q, scale=s)
+        byts = M * K * 3 + s.numel() * 4
+    elif case == "rmsnorm_quant":
+        M, H = 16384, 4096
+        x = rnd(M, H); gm = (torch.rand(H, device=dev, generator=g) + 0.5).to(torch.bfloat16)
+        q = torch.empty(M, H, dtype=torch.float8_e4m3fn, device=dev); s = torch.empty(M, device=dev)
+        f = lambda: w8.w8_rmsnorm_quant(x, gm, 1e-6, q=q, scale=s)
+        byts = M * H * 3 + H * 2 + M * 4
+    elif case == "silu_mul_quant":
+        M, I = 4096, 12288
+        x = rnd(M, 2 * I)
+        q = torch.empty(M, I, dtype=torch.float8_e4m3fn, device=dev); s = torch.empty(M, device=dev)
+        f = lambda: w8.w8_silu_mul_quant(x, q=q, scale=s)
+        byts = M * I * 5 + M * 4
+    elif case == "qk_norm_rope":
+        T, Hq, Hkv, D = 16384, 32, 8, 128
+        x = rnd(T, (Hq + 2 * Hkv) * D)
+        qw = (torch.rand(D, device=dev, generator=g) + 0.5).to(torch.bfloat16); kw = qw.clone()
+        pos = torch.randint(0, 8192, (T,), device=dev, generator=g)
+        ang = torch.rand(8192, D // 2, device=dev, generator=g) * 6.283
+        table = torch.cat([ang.cos(), ang.sin()], dim=1).float()
+        f = lambda: w8.w8_qk_norm_rope(x, Hq, Hkv, D, qw, kw, table, pos, out=x)
+        byts = T * (Hq + Hkv) * D * 4 + T * D * 4 + T * 8
+    elif case in ("gemm_fp8", "gemm_int8", "gemm_block"):
+        K, N, M = (4096, 24576, 8) if case != "gemm_block" else (5120, 51200, 8)
+        fmt = {"gemm_fp8": 0, "gemm_int8": 1, "gemm_block": 2}[case]
+        wb = rnd(N, K, scale=0.02)
+        if fmt == 2:
+            Wq, sW = w8.w8_quant_weight_block(wb)
+            A, sA = w8.w8_quant_per_token(rnd(M, K), w8.W8_Q_FP8, group=128)
+        else:
+            qf = w8.W8_Q_INT8 if fmt == 1 else w8.W8_Q_FP8
+            Wq, sW = w8.w8_quant_per_token(wb, qf)
+            A, sA = w8.w8_quant_per_token(rnd(M, K), qf)
+        del wb
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = w8.Workspace(dev)
+        f = lambda: w8.w8_gemm(fmt, A, sA, Wq, sW, out=out, workspace=ws)
+        byts = N * K + sW.numel() * 4 + M * K + sA.numel() * 4 + M * N * 2
+        flops = 2 * M * N * K
+    elif case == "grouped":
+        E, N, K, M, top = 128, 1536, 2048, 4, 8
+        wb = rnd(E * N, K, scale=0.02)
+        Wq, sW = w8.w8_quant_per_token(wb, w8.W8_Q_FP8); del wb
+        choice = torch.stack([torch.randperm(E, device=dev, generator=g)[:top] for _ in range(M)]).flatten()
+        counts = torch.bincount(choice, minlength=E)
+        off = torch.zeros(E + 1, dtype=torch.int32, device=dev); off[1:] = torch.cumsum(counts, 0).to(torch.int32)
+        A, sA = w8.w8_quant_per_token(rnd(M * top, K), w8.W8_Q_FP8)
+        out = torch.empty(M * top, N, dtype=torch.bfloat16, device=dev)
+        ws = w8.Workspace(dev)
+        f = lambda: w8.w8_grouped_gemm(0, A, sA, Wq.view(E, N, K), sW.view(E, N), off, max_tokens_per_expert=M,
+                                       out=out, workspace=ws)
+        used = int((counts > 0).sum().item())
+        byts = used * N * (K + 4) + M * top * (K + 4) + M * top * N * 2
+        flops = 2 * M * top * N * K
+    elif case == "pair_prefill":
+        M, K, N = 4096, 4096, 24576
+        A, sA = w8.w8_quant_per_token(rnd(M, K), w8.W8_Q_FP8)
+        Wq, sW = w8.w8_quant_per_token(rnd(N, K, scale=0.02), w8.W8_Q_FP8)
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = w8.Workspace(dev)
+        f = lambda: w8.w8_gemm(0, A, sA, Wq, sW, out=out, workspace=ws)
+        byts = M * K + N * K + (M + N) * 4 + M * N * 2
+        flops = 2 * M * N * K
+    else:
+        raise SystemExit("unknown kernel case %r (one of: %s)" % (case, ", ".join(KERNEL_CASES)))
+    return f, byts, flops
+
+
+def _flush_l2(dev):
+    import torch
+    # write a buffer larger than L2 so the next launch reads its inputs from HBM
+    torch.empty(256 << 20, dtype=torch.uint8, device=dev).fill_(1)
+
+
+def run_kernel_case(case):
+    """One hot-path kernel on its profiling-sized case (kernel_case), launched three times
+    with a write larger than the L2 before each (for `ncu -k <kernel> -s 2 -c 1`)."""
+    import torch
+    from bit_quantized_gemm_token_b200 import w8
+    if case not in KERNEL_CASES:
+        raise SystemExit("unknown kernel case %r (one of: %s)" % (case, ", ".join(KERNEL_CASES)))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    g = torch.Generator(device=dev); g.manual_seed(5)
+    f, _, _ = kernel_case(case, dev, g)
+    for _ in range(3):
+        _flush_l2(dev)
+        torch.cuda.synchronize()
+        f()
+        torch.cuda.synchronize()
+    assert w8.w8_device_status(1) == 0
+    print(json.dumps({"kernel_case": case, "launches": 3}))
+
+
+def time_kernels(dev, peak, tflops_peak, reps=7):
+    """Each hot-path kernel alone on its profiling-sized case (kernel_case): the median of
+    `reps` launches, each timed with CUDA events on the launching stream after a write
+    larger than the L2; HBM fraction (algorithmic bytes / time over the measured copy
+    peak) and, for the contractions, the tensor fraction of the bf16 peak times 2 (fp8 and
+    int8 run at twice the bf16 rate)."""
+    import torch
+    g = torch.Generator(device=dev); g.manual_seed(5)
+    res = {}
+    for case in KERNEL_CASES:
+        f, byts, flops = kernel_case(case, dev, g)
+        f()
+        torch.cuda.synchronize()
+        s = torch.cuda.current_stream()
+        ts = []
+        for _ in range(reps):
+            _flush_l2(dev)
+            e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(s); f(); e1.record(s)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        us = sorted(ts)[len(ts) // 2]
+        r = {"us": round(us, 2), "GB/s": round(byts / (us * 1e-6) / 1e9, 1),
+             "hbm_frac": round(byts / (us * 1e-6) / 1e9 / peak, 4), "bytes": byts}
+        if flops and tflops_peak:
+            r["TFLOP/s"] = round(flops / (us * 1e-6) / 1e12, 1)
+            r["tensor_frac"] = round(flops / (us * 1e-6) / 1e12 / (2 * tflops_peak), 4)
+        res[case] = r
+        del f
+        torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -848,12 +1071,19 @@ def main():
     ap.add_argument("--single", default="", help="KxN: time one shape only (profiling case)")
     ap.add_argument("--m", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-extras", action="store_true", help="skip timing the qk-norm/rope and grouped kernels")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip timing the other kernels (qk-norm/rope, grouped, the per-kernel table)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-table", action="store_true", help="skip the per-(format, shape, M) decode table")
+    ap.add_argument("--kernel", default="", help="run one kernel on its profiling case instead (for ncu): " +
+                    ", ".join(KERNEL_CASES))
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-seconds", type=float, default=3.0)
     args = ap.parse_args()
+    if args.kernel:
+        run_kernel_case(args.kernel)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

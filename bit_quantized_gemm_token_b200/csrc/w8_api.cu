@@ -323,6 +323,23 @@ int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int M, int
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
+int w8_gemm_timeout_debug(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
+                          void* out, int M, int N, int K, int variant, int wait_us, w8_stream_t stream)
+{
+    if (!A_q || !W_q || !out || !A_scale || !W_scale) return W8_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || wait_us < 1 || wait_us > 1000000) return W8_ERR_INVALID_ARG;
+    if (!aligned(A_q, 16) || !aligned(W_q, 16) || !aligned(out, 2)) return W8_ERR_ALIGNMENT;
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc != W8_OK) return rc;
+    GemmPlan plan;
+    rc = resolve(fmt, M, N, K, variant, sms, &plan);
+    if (rc < 0) return rc;
+    if (!plan.decode) return W8_ERR_UNSUPPORTED;
+    return gemm_launch(plan, A_q, A_scale, W_q, W_scale, out, nullptr, nullptr, 0, reinterpret_cast<cudaStream_t>(stream),
+                       nullptr, 1, (unsigned long long)wait_us * 1000ull);
+}
+
 int w8_gemm_resolve_variant(int fmt, int M, int N, int K, int variant)
 {
     int sms = 0;
@@ -470,8 +487,8 @@ int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, c
     if (!qkv || !out || !q_weight || !k_weight || !cos_sin || !positions) return W8_ERR_INVALID_ARG;
     if (T < 0 || Hq < 0 || Hkv < 0 || max_pos <= 0 || !(eps >= 0.0f)) return W8_ERR_INVALID_ARG;
     if (D != 64 && D != 128 && D != 256) return W8_ERR_UNSUPPORTED;
-    if (!aligned(qkv, 8) || !aligned(out, 8) || !aligned(q_weight, 8) || !aligned(k_weight, 8) || !aligned(cos_sin, 4) ||
-        !aligned(positions, 8))
+    if (!aligned(qkv, 16) || !aligned(out, 16) || !aligned(q_weight, 16) || !aligned(k_weight, 16) ||
+        !aligned(cos_sin, 16) || !aligned(positions, 8))
         return W8_ERR_ALIGNMENT;
     int rc = check_device(nullptr);
     if (rc != W8_OK) return rc;

@@ -51,13 +51,82 @@ __device__ __forceinline__ uint32_t int8_code(float v)
     return static_cast<uint32_t>(r) & 0xFFu;
 }
 
-// 8 values / s -> 8 codes packed little-endian into a uint2.
+// Correctly rounded x / s for the quantizers, without a division per element.  The row's
+// divisor is prepared once: y = RN(1 / s') with s' = s, or s * 2^64 when s is below 2^-92
+// (x is scaled by the same exact power of two).  Per element (Markstein's theorem,
+// P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990; J.-M. Muller et al., "Handbook of
+// Floating-Point Arithmetic", ch. on division with an FMA):
+//   q0 = RN(x * y);  r = x - q0 * s' (one fma);  q = RN(q0 + r * y)
+// is the correctly rounded quotient whenever the remainder r is exact.  r is a multiple
+// of ulp(q0) ulp(s'), so it is an fp32 value when that product is at least 2^-149: with
+// s' >= 2^-92 this holds for every |q0| >= 2^-10, and smaller quotients give a zero code
+// in both formats (e4m3 rounds values up to 2^-10 to zero, int8 values below 1/2).  So
+// the codes, and the quotient wherever a code can depend on it, are those of IEEE
+// division; the sign of x is copied onto q so that -0 stays -0.  Checked on the device
+// against __fdiv_rn (w8_selfcheck.cu): every bf16 x with every bf16 amax, infinities
+// included, |x| <= amax (amax / 448, amax / 127, UE8M0), and 2^30 fp32 numerators per
+// scale rule, half of them within a few ulps of a code's rounding boundary.
+struct RowDivisor {
+    float s;      // s' (s, or s * 2^64)
+    float y;      // RN(1 / s')
+    float f;      // 1, or 2^64: the factor applied to x
+    bool plain;   // f = 1 and no element of the row is infinite: quotient_plain applies
+};
+
+__device__ __forceinline__ RowDivisor make_divisor(float s)
+{
+    RowDivisor d;
+    const bool tiny = s < 0x1p-92f;
+    d.f = tiny ? 0x1p64f : 1.0f;
+    d.s = __fmul_rn(s, d.f);
+    d.y = __frcp_rn(d.s);
+    // s = +inf (an infinite amax): y = 0, and s' = 0 keeps the correction finite, so a
+    // finite x gives +-0 and an infinite x NaN, as x / inf does
+    if (isinf(s)) d.s = 0.0f;
+    d.plain = false;
+    return d;
+}
+
+// The same divisor for a row (or group) whose maximum magnitude amax is known: when no
+// scaling is needed and amax is finite (so no element is infinite and q0 never is),
+// quotient_plain gives quotient_rn's result with two operations fewer per element.
+__device__ __forceinline__ RowDivisor make_divisor(float s, float amax)
+{
+    RowDivisor d = make_divisor(s);
+    d.plain = d.f == 1.0f && isfinite(amax) && !isinf(s);
+    return d;
+}
+
+__device__ __forceinline__ float quotient_rn(float x, const RowDivisor& d)
+{
+    const float xs = __fmul_rn(x, d.f);
+    const float q0 = __fmul_rn(xs, d.y);
+    const float r = __fmaf_rn(-q0, d.s, xs);
+    // an infinite q0 comes only from an infinite x over a finite s: the quotient is q0
+    return copysignf(fabsf(q0) == INFINITY ? q0 : __fmaf_rn(r, d.y, q0), x);
+}
+
+// quotient_rn for a divisor with d.plain set (x finite or NaN, no scaling)
+__device__ __forceinline__ float quotient_plain(float x, const RowDivisor& d)
+{
+    const float q0 = __fmul_rn(x, d.y);
+    const float r = __fmaf_rn(-q0, d.s, x);
+    return copysignf(__fmaf_rn(r, d.y, q0), x);
+}
+
+// 8 values / s -> 8 codes packed little-endian into a uint2 (d = make_divisor(s)).
 template <int QFMT>
-__device__ __forceinline__ uint2 encode8(const float (&f)[8], float s)
+__device__ __forceinline__ uint2 encode8(const float (&f)[8], const RowDivisor& d)
 {
     float v[8];
+    if (d.plain) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fdiv_rn(f[i], s);
+        for (int i = 0; i < 8; ++i) v[i] = quotient_plain(f[i], d);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = quotient_rn(f[i], d);
+    }
     uint2 r;
     if (QFMT == W8_Q_FP8) {
         r.x = e4m3x2(v[0], v[1]) | (e4m3x2(v[2], v[3]) << 16);
@@ -79,42 +148,6 @@ __device__ __forceinline__ float scale_from_amax(float amax, float qmax, bool ue
     int p = (f == 0.5f) ? e - 1 : e;  // smallest power of two >= r
     p = max(-127, min(127, p));
     return ldexpf(1.0f, p);
-}
-
-// Correctly rounded x / s for the quantizers, without a division per element.  The row's
-// divisor is prepared once: y = RN(1 / s') with s' = s (or s * 2^64 when s is below 2^-100,
-// so that 1 / s' stays finite; x is scaled by the same exact power of two).  Per element
-// (Markstein's theorem, P. Markstein, "Computation of elementary functions on the IBM
-// RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; J.-M. Muller et al.,
-// "Handbook of Floating-Point Arithmetic", ch. on division with an FMA):
-//   q0 = RN(x * y);  r = x - q0 * s' (exact, one fma);  q = RN(q0 + r * y)
-// is the correctly rounded quotient while q stays in the normal range; the sign of x is
-// copied onto q so that -0 stays -0.  Outside the normal range (|q| < 2^-126) q may differ
-// from RN(x / s) in its last bits, but every such value encodes to a zero code.  Checked
-// against __fdiv_rn for every bf16 x and every bf16 amax with |x| <= amax (amax / 448,
-// amax / 127, UE8M0): identical e4m3 and int8 codes.
-struct RowDivisor {
-    float s;    // s' (s, or s * 2^64)
-    float y;    // RN(1 / s')
-    float f;    // 1, or 2^64: the factor applied to x
-};
-
-__device__ __forceinline__ RowDivisor make_divisor(float s)
-{
-    RowDivisor d;
-    const bool tiny = s < 0x1p-100f;
-    d.f = tiny ? 0x1p64f : 1.0f;
-    d.s = __fmul_rn(s, d.f);
-    d.y = __frcp_rn(d.s);
-    return d;
-}
-
-__device__ __forceinline__ float quotient_rn(float x, const RowDivisor& d)
-{
-    const float xs = __fmul_rn(x, d.f);
-    const float q0 = __fmul_rn(xs, d.y);
-    const float r = __fmaf_rn(-q0, d.s, xs);
-    return copysignf(__fmaf_rn(r, d.y, q0), x);
 }
 
 }  // namespace w8

@@ -178,19 +178,21 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
         return W8_OK;
     }
     if (variant & W8_V_PAIR) {
-        // 256 x 256 tiles on CTA pairs: Standard full-K loop, FP8-dynamic / INT8
-        if (block || q.swap || q.stream || lg != 0 || q.cluster || q.bm != 128 || q.pfix || tid != kTileBN256 ||
+        // 256 x 256 tiles on CTA pairs: Standard full-K loop, FP8-dynamic / INT8; with a
+        // K split, one (tile, K chunk) unit per pair
+        if (block || q.swap || q.stream || lg > 3 || q.cluster || q.bm != 128 || q.pfix || tid != kTileBN256 ||
             kps > 1)
             return W8_ERR_UNSUPPORTED;
         if (stages == 0) stages = 5;   // measured: 5 a little ahead of 6 at M = 4096
         if (stages < 2) return W8_ERR_UNSUPPORTED;
         q.pair = 1;
         q.bn = 256;
-        q.split = 1;
+        q.split = 1 << lg;
         q.kps = 1;
         q.stages = stages;
         q.kbs = (K + 127) / 128;
         q.nsb = q.kbs;
+        if (q.split > q.kbs) return W8_ERR_UNSUPPORTED;
         q.smem_bytes = 1024 + (size_t)stages * 2 * 128 * 128 + (size_t)(2 * stages + 5) * 8 + 16;
         if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
         q.rows_R = M;
@@ -200,6 +202,18 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
         q.tiles = q.r_tiles * q.c_tiles;
         q.units = (long long)q.tiles * q.nsb;
         const long long pairs_max = (sm_count > 0 ? sm_count : 148) / 2;
+        if (q.split > 1) {
+            // one unit per pair, every pair resident at once; a workspace slot of 128 x 256
+            // words per CTA and a ticket counter per half-tile
+            const long long units = (long long)q.tiles * q.split;
+            if (units > pairs_max || 2LL * q.tiles > kMaxCounterTiles) return W8_ERR_UNSUPPORTED;
+            q.G = (int)(2 * units);
+            q.align_tiles = 1;
+            q.ws_counters = (size_t)kMaxCounterTiles * 4;
+            q.ws_bytes = q.ws_counters + (size_t)units * 2 * 256 * 128 * 4;
+            *p = q;
+            return W8_OK;
+        }
         const long long pairs = q.tiles < pairs_max ? q.tiles : pairs_max;
         if (pairs < 1) return W8_ERR_UNSUPPORTED;
         q.G = (int)(2 * pairs);
@@ -288,7 +302,8 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
 
 // ---------------------------------------------------------------- launch
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
-                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s, const int* g_off)
+                void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s, const int* g_off,
+                int starve, unsigned long long wait_ns)
 {
     if (p.ws_bytes > 0 && (workspace == nullptr || ws_bytes < p.ws_bytes)) return W8_ERR_WORKSPACE;
     if (p.ws_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return W8_ERR_ALIGNMENT;
@@ -322,6 +337,8 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
         args.nkb_lo = p.nkb_lo;
         args.recv_first[0] = p.recv_first[0];
         args.recv_first[1] = p.recv_first[1];
+        args.starve = starve;
+        args.wait_ns = wait_ns;
         const cudaError_t e = launch_decode(p, maps, args, s);
         if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
         return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
@@ -344,7 +361,7 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
     args.units = p.units;
     args.G = p.G;
     args.align_tiles = p.align_tiles;
-    args.csplit = p.cluster ? p.split : 0;
+    args.csplit = (p.cluster || p.pair) ? p.split : 0;
     args.pfix = p.pfix;
     args.grouped = p.grouped;
     args.g_E = p.g_E;
@@ -467,7 +484,7 @@ int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, co
     args.units = p.units;
     args.G = p.G;
     args.align_tiles = p.align_tiles;
-    args.csplit = p.cluster ? p.split : 0;
+    args.csplit = (p.cluster || p.pair) ? p.split : 0;
     args.w_ptr = static_cast<const uint8_t*>(W_q);
     args.stages = p.stages;
     args.pdl = p.pdl;

@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     // width of rank r's column share
     auto share = [&](int r) { return max(0, min(SW, BN - r * SW)); };
     const uint32_t tmem_cols = tmem_cols_for(BN);
+    const uint64_t wlim = a.wait_ns ? a.wait_ns : kWaitNs;   // bound on every wait
+    const int nload = a.starve ? 0 : nkb;                     // K blocks the producer loads
     // Receive area: [C source ranks][M tokens][RS words], the partial sums of the columns
     // this rank finishes.  It lies over the R consecutive stages whose last use comes
     // earliest, so that it is free -- and the other ranks may write into it -- a few K
@@ -173,27 +175,27 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int D = a.l2ahead;
             // weights are never written by the work ahead of this kernel: under PDL the
             // first stages' weight boxes are requested before waiting for it
-            const int pre = a.pdl ? min(nkb, S) : 0;
+            const int pre = a.pdl ? min(nload, S) : 0;
             for (int i = 0; i < pre; ++i) {
                 const uint32_t fb = ptx::smem_u32(full + i);
                 ptx::mbar_arrive_expect_tx(fb, tx);
                 ptx::tma_load_2d(ptx::smem_u32(w_slot(i)), &tmW, fb, (kb0 + i) * 128, n0, pol_w);
             }
-            const int first = min(nkb, S);   // K blocks whose loads go out without waiting for a stage
-            for (int i = first; i < min(nkb, first + D); ++i) ptx::tma_prefetch_l2_2d(&tmW, (kb0 + i) * 128, n0);
+            const int first = min(nload, S);   // K blocks whose loads go out without waiting for a stage
+            for (int i = first; i < min(nload, first + D); ++i) ptx::tma_prefetch_l2_2d(&tmW, (kb0 + i) * 128, n0);
             ptx::grid_dep_wait();
             for (int i = 0; i < pre; ++i)
                 ptx::tma_load_2d(ptx::smem_u32(a_slot(i)), &tmA, ptx::smem_u32(full + i), (kb0 + i) * 128, 0, pol_a);
             int stage = pre % S;
             uint32_t phase = (pre == S) ? 1u : 0u;
             int issued = pre;
-            for (int i = pre; i < nkb; ++i) {
-                if (!wait_bounded(ptx::smem_u32(empty + stage), phase ^ 1u, abort_flag)) break;
+            for (int i = pre; i < nload; ++i) {
+                if (!wait_bounded(ptx::smem_u32(empty + stage), phase ^ 1u, abort_flag, wlim)) break;
                 const uint32_t fb = ptx::smem_u32(full + stage);
                 ptx::mbar_arrive_expect_tx(fb, tx);
                 ptx::tma_load_2d(ptx::smem_u32(w_slot(stage)), &tmW, fb, (kb0 + i) * 128, n0, pol_w);
                 ptx::tma_load_2d(ptx::smem_u32(a_slot(stage)), &tmA, fb, (kb0 + i) * 128, 0, pol_a);
-                if (i >= first && i + D < nkb) ptx::tma_prefetch_l2_2d(&tmW, (kb0 + i + D) * 128, n0);
+                if (i >= first && i + D < nload) ptx::tma_prefetch_l2_2d(&tmW, (kb0 + i + D) * 128, n0);
                 ++issued;
                 if (++stage == S) { stage = 0; phase ^= 1u; }
             }
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 bool free_ok = true;
                 for (int st = s0; st < s0 + R && free_ok; ++st) {
                     const int j = last_use(st, nkb);
-                    if (j >= 0) free_ok = wait_bounded(ptx::smem_u32(empty + st), (uint32_t)((j / S) & 1), abort_flag);
+                    if (j >= 0) free_ok = wait_bounded(ptx::smem_u32(empty + st), (uint32_t)((j / S) & 1), abort_flag, wlim);
                 }
                 if (free_ok)
                     for (int r = 0; r < C; ++r)
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t phase = 0;
             bool ok = true;
             for (int i = 0; i < nkb; ++i) {
-                ok = wait_bounded(ptx::smem_u32(full + stage), phase, abort_flag);
+                ok = wait_bounded(ptx::smem_u32(full + stage), phase, abort_flag, wlim);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const uint64_t dA = smem_desc(ptx::smem_u32(a_slot(stage)));
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (te < M) sa_r = __ldg(a.sA + te);
         }
-        bool ok = wait_bounded(ptx::smem_u32(tfull), 0, abort_flag);
+        bool ok = wait_bounded(ptx::smem_u32(tfull), 0, abort_flag, wlim);
         if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !ok)) ok = false;
         ptx::tc_fence_after();
         const uint32_t recvb_s = ptx::smem_u32(recvb);
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         };
         auto wait_free = [&]() {
             // every other rank's receive area is free
-            const bool f = wait_bounded<true>(ptx::smem_u32(freeb), 0, abort_flag);
+            const bool f = wait_bounded<true>(ptx::smem_u32(freeb), 0, abort_flag, wlim);
             if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !f)) ok = false;
         };
         if (ok && use_stg) {
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // this rank's own partials and the scales are in place; then the others' partials
         ptx::bar_sync(kEpiBarrier, kEpiThreads);
         if (ok && C > 1) {
-            const bool g = wait_bounded<true>(ptx::smem_u32(recvb), 0, abort_flag);
+            const bool g = wait_bounded<true>(ptx::smem_u32(recvb), 0, abort_flag, wlim);
             if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !g)) ok = false;
         }
         // every exchange with the other ranks is over (what this rank sent has landed in

@@ -108,6 +108,10 @@ struct GemmArgs {
     int recv_R;           // stages spanned by a rank's receive area
     int nkb_lo;           // the smaller of the two K-block counts a rank holds
     int recv_first[2];    // first stage of the receive area for nkb_lo and nkb_lo + 1 K blocks
+    // failure-path check (w8_gemm_timeout_debug): the producer issues no loads and every
+    // wait gives up after wait_ns (0: the normal bound)
+    int starve;
+    unsigned long long wait_ns;
 };
 
 // K blocks a CTA with units [u0, u1) multiplies: its own range when the units lie in one
@@ -185,7 +189,8 @@ __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_sta
 // Poll an mbarrier phase until it completes, the deadline passes, or another role of
 // this CTA has given up (abort flag).  Returns false on give-up.
 template <bool CLUSTER_SCOPE = false>
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag)
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                             uint64_t limit_ns = kWaitNs)
 {
     auto probe = [&] { return CLUSTER_SCOPE ? ptx::mbar_try_wait_cluster(bar, parity) : ptx::mbar_try_wait(bar, parity); };
     if (probe()) return true;
@@ -194,7 +199,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
         if (probe()) return true;
         if ((it & 255u) == 0) {
             if (*abort_flag) return false;
-            if (ptx::globaltimer_ns() - t0 > kWaitNs) {
+            if (ptx::globaltimer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 record_error(W8_ERR_DEVICE_TIMEOUT);
                 return false;

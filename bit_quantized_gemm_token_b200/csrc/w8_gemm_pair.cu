@@ -15,6 +15,14 @@
 //     tensor memory; the commits arrive on the stage and accumulator barriers of both;
 //   * each CTA's epilogue scales and stores its own 128 token rows, then tells the
 //     leader (remote arrive for rank 1) that the accumulator may be reused.
+// Split-K (split S = 2..8, a power of two): pair p computes K chunk p % S (contiguous K
+// blocks [c kbs / S, (c + 1) kbs / S)) of tile p / S, one unit per pair, so the grid has
+// 2 tiles S CTAs (at most one per SM pair).  Each CTA publishes its 128 x 256 partial
+// sums to its own workspace slot ([column][row] words), takes a ticket on its half-tile's
+// counter, and the last of the S contributors adds the S slots in chunk order -- a fixed
+// order, so results do not depend on which finishes last -- then scales and stores, and
+// resets the counter for the next call.  This fills the chip when a few tall tiles carry
+// a long K (the down projection at a few hundred tokens: 16 tiles of K = 12288).
 // Every wait is bounded (1 s, abort flag, device status W8_ERR_DEVICE_TIMEOUT).  No load
 // uses cluster multicast.
 #include "w8_gemm_kernel.cuh"
@@ -107,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* ticket = reinterpret_cast<volatile int*>(tmem_slot + 2);
     auto a_slot = [&](int s) { return smem + (size_t)s * kPairStage; };
     auto b_slot = [&](int s) { return smem + (size_t)s * kPairStage + kHalfBytes; };
 
@@ -145,12 +154,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem = *tmem_slot;
     }
 
-    // pair p (the cluster) takes the tiles [p T / P, (p + 1) T / P), weight tile fastest
+    // pair p (the cluster) takes the tiles [p T / P, (p + 1) T / P), weight tile fastest;
+    // with a K split, the K chunk p % S of tile p / S
     const int P = (int)(gridDim.x >> 1);
     const int pr = (int)(blockIdx.x >> 1);
     const int T = a.tiles;
-    const int t0 = (int)((long long)pr * T / P), t1 = (int)((long long)(pr + 1) * T / P);
-    const int kbs = a.kbs;
+    const int S_k = a.csplit > 1 ? a.csplit : 1;
+    const int t0 = S_k > 1 ? pr / S_k : (int)((long long)pr * T / P);
+    const int t1 = S_k > 1 ? t0 + 1 : (int)((long long)(pr + 1) * T / P);
+    const int chunk = S_k > 1 ? pr % S_k : 0;
+    const int kb0 = (int)((long long)chunk * a.kbs / S_k), kb1 = (int)((long long)(chunk + 1) * a.kbs / S_k);
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -165,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = t0; t < t1 && ok; ++t) {
                 const int rt = t / a.c_tiles, ct = t % a.c_tiles;
                 const int ya = rt * 256 + (int)rank * 128, yb = ct * 256 + (int)rank * 128;
-                for (int kb = 0; kb < kbs; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!wait_bounded(ptx::smem_u32(empty + stage), phase ^ 1u, abort_flag)) { ok = false; break; }
                     const uint32_t fb = ptx::map_to_rank(ptx::smem_u32(full + stage), 0);
                     if (rank == 0) ptx::mbar_arrive_expect_tx(ptx::smem_u32(full + stage), 2u * kPairStage);
@@ -210,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = wait_bounded<true>(ptx::smem_u32(tempty + buf), bphase ^ 1u, abort_flag);
                     ptx::tc_fence_after();
                     const uint32_t d_tmem = tmem + (uint32_t)(buf * 256);
-                    for (int kb = 0; kb < kbs && ok; ++kb) {
+                    for (int kb = kb0; kb < kb1 && ok; ++kb) {
                         ok = wait_bounded(ptx::smem_u32(full + stage), phase, abort_flag);
                         if (!ok) break;
                         ptx::tc_fence_after();
@@ -218,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t dB = smem_desc(ptx::smem_u32(b_slot(stage)));
 #pragma unroll
                         for (int k = 0; k < 4; ++k)   // 32 K-bytes per MMA: +2 in 16-byte units
-                            mma_pair<KIND>(d_tmem, dA + 2 * k, dB + 2 * k, kIdesc, (kb == 0 && k == 0) ? 0u : 1u);
+                            mma_pair<KIND>(d_tmem, dA + 2 * k, dB + 2 * k, kIdesc, (kb == kb0 && k == 0) ? 0u : 1u);
                         commit_pair(ptx::smem_u32(empty + stage), 0x3);
                         if (++stage == S) { stage = 0; phase ^= 1u; }
                     }
@@ -238,7 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ epilogue (both CTAs)
         ptx::grid_dep_wait();
         const int i = (warp & 3) * 32 + lane;   // accumulator row (TMEM lane) of this thread
+        const int te = threadIdx.x - 64;        // 0 .. 127 over the epilogue warps
         const uint32_t t_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        constexpr size_t kSlotWords = 256 * 128;
         int buf = 0;
         uint32_t bphase = 0;
         for (int t = t0; t < t1; ++t) {
@@ -250,12 +265,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool has_row = r_row < a.M;
             const float s_row = (has_row && a.out_i32 == nullptr) ? __ldg(a.sA + r_row) : 1.0f;
             const int c_base = ct * 256;
+            if (S_k == 1) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 16) {
-                if (c_base + c0 >= a.N) break;
-                uint32_t v[16];
-                ptx::tmem_ld16(t_lane + (uint32_t)(buf * 256 + c0), v);
-                if (has_row) store_chunk16<KIND, false>(a, a.sA, r_row, c_base + c0, v, s_row);
+                for (int c0 = 0; c0 < 256; c0 += 16) {
+                    if (c_base + c0 >= a.N) break;
+                    uint32_t v[16];
+                    ptx::tmem_ld16(t_lane + (uint32_t)(buf * 256 + c0), v);
+                    if (has_row) store_chunk16<KIND, false>(a, a.sA, r_row, c_base + c0, v, s_row);
+                }
+            } else {
+                // publish this CTA's partial sums: [column][row] words, 512 contiguous bytes
+                // per column over the 128 threads
+                uint32_t* my = a.partials + ((size_t)pr * 2 + rank) * kSlotWords;
+#pragma unroll 1
+                for (int c0 = 0; c0 < 256; c0 += 16) {
+                    if (c_base + c0 >= a.N) break;
+                    uint32_t v[16];
+                    ptx::tmem_ld16(t_lane + (uint32_t)(buf * 256 + c0), v);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) __stcg(my + (size_t)(c0 + jj) * 128 + i, v[jj]);
+                }
             }
             ptx::tc_fence_before();
             __syncwarp();
@@ -264,6 +293,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                 else ptx::mbar_arrive_remote(ptx::map_to_rank(ptx::smem_u32(tempty + buf), 0));
             }
             if (++buf == 2) { buf = 0; bphase ^= 1u; }
+            if (S_k > 1) {
+                // ticket on this half-tile's counter: the last contributor finishes it
+                __threadfence();
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (te == 0) *ticket = atomicAdd(a.counters + t * 2 + (int)rank, 1);
+                ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                if (*ticket == S_k - 1) {
+                    __threadfence();
+#pragma unroll 1
+                    for (int c0 = 0; c0 < 256; c0 += 16) {
+                        if (c_base + c0 >= a.N) break;
+                        uint32_t v[16];
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) v[jj] = 0u;
+                        // the S chunks' partials in chunk order, four in flight together
+#pragma unroll 1
+                        for (int cb = 0; cb < S_k; cb += 4) {
+                            uint32_t x[4][16];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                if (cb + k < S_k) {
+                                    const uint32_t* p = a.partials + ((size_t)(t * S_k + cb + k) * 2 + rank) * kSlotWords +
+                                                        (size_t)c0 * 128 + i;
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj) x[k][jj] = __ldcg(p + (size_t)jj * 128);
+                                }
+                            }
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                if (cb + k < S_k)
+#pragma unroll
+                                    for (int jj = 0; jj < 16; ++jj)
+                                        v[jj] = (cb + k == 0) ? x[k][jj] : add_words<KIND>(v[jj], x[k][jj]);
+                        }
+                        if (has_row) store_chunk16<KIND, false>(a, a.sA, r_row, c_base + c0, v, s_row);
+                    }
+                    if (te == 0) a.counters[t * 2 + (int)rank] = 0;   // ready for the next call
+                }
+            }
         }
     }
 

@@ -70,9 +70,10 @@ struct GemmPlan {
 };
 
 int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p);
+// starve / wait_ns (decode form only): the failure-path check of w8_gemm_timeout_debug
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                 void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s,
-                const int* g_off = nullptr);
+                const int* g_off = nullptr, int starve = 0, unsigned long long wait_ns = 0);
 int gemm_occupancy(const GemmPlan& p, int* n);
 int launch_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
                         const void* k_weight, const float* cos_sin, int max_pos, const long long* positions, float eps,

@@ -9,13 +9,12 @@
 //   with c_i, s_i the cosine / sine row of the token's position (table input,
 //   fp32 [max_pos, D]: cosines then sines), each pair (y_i, y_{i+D/2}) is rotated:
 //   o_i = y_i c_i - y_{i+D/2} s_i,  o_{i+D/2} = y_{i+D/2} c_i + y_i s_i  (fp32), -> bf16.
-// Value heads are copied (or left in place).  One warp per four consecutive heads of a
-// token (their loads issued together); lane l holds the D/64 consecutive elements
-// l*D/64.. of each half of every head, so every rotated pair is in one thread.  HBM-bound:
-// each head is read once and written once.
+// Value heads are copied (or left in place).  D / 16 lanes share a head: lane s of the
+// head's group holds the 8 consecutive elements 8s.. of each half (one 16-byte vector per
+// half), so every rotated pair is in one thread and a warp covers 512 / D consecutive heads
+// of a token at once; each warp takes G such groups, their loads all issued before any
+// arithmetic.  HBM-bound: each head is read once and written once.
 #include <cuda_bf16.h>
-
-#include <type_traits>
 
 #include "w8_internal.h"
 #include "w8_ptx.cuh"
@@ -26,100 +25,139 @@ namespace {
 
 static __device__ int g_qknr_status;
 
-// C = elements per lane per half (D = 64 C); HPW = heads per warp (one token's
-// consecutive heads: their loads are all in flight together, and the token's cos / sin
-// values are loaded once for them)
-template <int C, int HPW>
-__global__ void __launch_bounds__(128) qk_norm_rope_kernel(const __nv_bfloat16* __restrict__ qkv,
-                                                           __nv_bfloat16* __restrict__ out, int T, int Hq, int Hkv,
-                                                           const __nv_bfloat16* __restrict__ qw,
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);   // .x = a (low half), .y = b
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// D = head dimension (64, 128 or 256); G = head groups per warp; Hn = heads touched per
+// token (query + key heads in place, all heads otherwise); units = T * ceil(Hn / (512 / D))
+template <int D, int G>
+__global__ void __launch_bounds__(128, 8) qk_norm_rope_kernel(const __nv_bfloat16* __restrict__ qkv,
+                                                           __nv_bfloat16* __restrict__ out, int Hq, int Hkv, int Hn,
+                                                           int units, const __nv_bfloat16* __restrict__ qw,
                                                            const __nv_bfloat16* __restrict__ kw,
                                                            const float* __restrict__ cos_sin, int max_pos,
                                                            const long long* __restrict__ positions, float eps)
 {
     ptx::grid_dep_launch();
     ptx::grid_dep_wait();
-    constexpr int D = 64 * C, HALF = 32 * C;
+    constexpr int HALF = D / 2, LPH = D / 16, HPW = 32 / LPH;
+    // no term passes through more than 16 (the lane's fp64 chain) + log2(LPH) roundings
+    constexpr int kDepth = 16 + 5;
     const int H = Hq + 2 * Hkv;
-    const int groups = (H + HPW - 1) / HPW;
-    const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (wid >= (long long)T * groups) return;
-    const int lane = threadIdx.x & 31;
-    const int t = (int)(wid / groups), h0 = (int)(wid % groups) * HPW;
-    const int nh = min(HPW, H - h0);
-    // lane l: elements [l*C, l*C + C) of each half, as one C*2-byte vector
-    using Vec = typename std::conditional<C == 1, unsigned short, typename std::conditional<C == 2, unsigned int, uint2>::type>::type;
-    Vec lov[HPW], hiv[HPW];
+    const int groups = (Hn + HPW - 1) / HPW;
+    const int wid = (int)(((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * G);
+    if (wid >= units) return;
+    const int lane = threadIdx.x & 31, sub = lane % LPH;
+    uint4 lov[G], hiv[G];
+    int tt[G], hh[G];
+    bool act[G];
 #pragma unroll
-    for (int j = 0; j < HPW; ++j) {
-        if (j < nh) {
-            const __nv_bfloat16* x = qkv + ((size_t)t * H + h0 + j) * D;
-            lov[j] = *reinterpret_cast<const Vec*>(x + lane * C);
-            hiv[j] = *reinterpret_cast<const Vec*>(x + HALF + lane * C);
+    for (int g = 0; g < G; ++g) {
+        const int u = wid + g;
+        tt[g] = u / groups;
+        hh[g] = (u - tt[g] * groups) * HPW + lane / LPH;
+        act[g] = u < units && hh[g] < Hn;
+        if (act[g]) {
+            const __nv_bfloat16* x = qkv + ((size_t)tt[g] * H + hh[g]) * D + sub * 8;
+            lov[g] = *reinterpret_cast<const uint4*>(x);
+            hiv[g] = *reinterpret_cast<const uint4*>(x + HALF);
+        } else {
+            lov[g] = make_uint4(0, 0, 0, 0);
+            hiv[g] = make_uint4(0, 0, 0, 0);
         }
     }
-    const long long p = positions[t];
-    const bool pos_ok = p >= 0 && p < max_pos;
-    float cv[C], sv[C];
-    if (pos_ok && h0 < Hq + Hkv) {
-        const float* cs = cos_sin + (size_t)p * D;
+    long long pos[G];
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            cv[i] = __ldg(cs + lane * C + i);
-            sv[i] = __ldg(cs + HALF + lane * C + i);
-        }
-    }
-    if (!pos_ok && h0 < Hq + Hkv && lane == 0) atomicCAS(&g_qknr_status, 0, W8_ERR_INVALID_ARG);
-    auto unpack = [](Vec v, float (&f)[C]) {
-        const unsigned short* b = reinterpret_cast<const unsigned short*>(&v);
+    for (int g = 0; g < G; ++g) pos[g] = act[g] && hh[g] < Hq + Hkv ? __ldg(positions + tt[g]) : 0;
 #pragma unroll
-        for (int i = 0; i < C; ++i) f[i] = __uint_as_float((uint32_t)b[i] << 16);
-    };
-#pragma unroll
-    for (int j = 0; j < HPW; ++j) {
-        if (j >= nh) break;
-        const int h = h0 + j;
-        __nv_bfloat16* o = out + ((size_t)t * H + h) * D;
-        if (h >= Hq + Hkv) {
+    for (int g = 0; g < G; ++g) {
+        const int h = hh[g];
+        const bool rot = act[g] && h < Hq + Hkv;
+        const bool pos_ok = pos[g] >= 0 && pos[g] < max_pos;
+        if (rot && !pos_ok && sub == 0) atomicCAS(&g_qknr_status, 0, W8_ERR_INVALID_ARG);
+        __nv_bfloat16* o = out + ((size_t)tt[g] * H + h) * D + sub * 8;
+        if (act[g] && !rot && out != qkv) {
             // value head: pass through
-            if (out != qkv) {
-                *reinterpret_cast<Vec*>(o + lane * C) = lov[j];
-                *reinterpret_cast<Vec*>(o + HALF + lane * C) = hiv[j];
+            *reinterpret_cast<uint4*>(o) = lov[g];
+            *reinterpret_cast<uint4*>(o + HALF) = hiv[g];
+        }
+        float lo[8], hi[8];
+        unpack8(lov[g], lo);
+        unpack8(hiv[g], hi);
+        // the exact sum of squares of the head, rounded once to fp32 (w8_sumsq.cuh); every
+        // lane of the warp runs the butterflies (inactive lanes hold zeros)
+        double ss64 = 0.0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            ss64 = __fma_rn((double)lo[i], (double)lo[i], ss64);
+            ss64 = __fma_rn((double)hi[i], (double)hi[i], ss64);
+        }
+#pragma unroll
+        for (int off = LPH / 2; off > 0; off >>= 1) ss64 = __dadd_rn(ss64, __shfl_xor_sync(0xFFFFFFFFu, ss64, off));
+        float ssf;
+        const bool sure = sq_round_certain(ss64, kDepth, &ssf);
+        if (__any_sync(0xFFFFFFFFu, !sure)) {
+            DSum ds{0.0, 0.0};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                ds = dsum_sq(ds, lo[i]);
+                ds = dsum_sq(ds, hi[i]);
             }
-            continue;
-        }
-        if (!pos_ok) continue;
-        float lo[C], hi[C];
-        unpack(lov[j], lo);
-        unpack(hiv[j], hi);
-        // the exact sum of squares rounded once to fp32 (w8_sumsq.cuh): lane sums, then the warp
-        DSum ss{0.0, 0.0};
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            ss = dsum_sq(ss, lo[i]);
-            ss = dsum_sq(ss, hi[i]);
+            for (int off = LPH / 2; off > 0; off >>= 1) ds = dsum_add(ds, dsum_shfl_xor(ds, off));
+            if (!sure) ssf = dsum_to_f32(ds);
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss = dsum_add(ss, dsum_shfl_xor(ss, off));
-        const float mean = __fdiv_rn(dsum_to_f32(ss), (float)D);
+        if (!rot || !pos_ok) continue;
+        const float* cs = cos_sin + (size_t)pos[g] * D + sub * 8;
+        const float4 c0 = __ldg(reinterpret_cast<const float4*>(cs));
+        const float4 c1 = __ldg(reinterpret_cast<const float4*>(cs + 4));
+        const float4 s0 = __ldg(reinterpret_cast<const float4*>(cs + HALF));
+        const float4 s1 = __ldg(reinterpret_cast<const float4*>(cs + HALF + 4));
+        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        // ss / D with D a power of two is an exact scaling (the same rounding as the quotient)
+        const float mean = __fmul_rn(ssf, 1.0f / D);
         const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
-        const __nv_bfloat16* w = (h < Hq) ? qw : kw;
-        float wl[C], wh[C];
-        unpack(*reinterpret_cast<const Vec*>(w + lane * C), wl);
-        unpack(*reinterpret_cast<const Vec*>(w + HALF + lane * C), wh);
-        unsigned short ol[C], oh[C];
+        const __nv_bfloat16* w = (h < Hq ? qw : kw) + sub * 8;
+        float wl[8], wh[8];
+        unpack8(__ldg(reinterpret_cast<const uint4*>(w)), wl);
+        unpack8(__ldg(reinterpret_cast<const uint4*>(w + HALF)), wh);
+        uint32_t ol[4], oh[4];
 #pragma unroll
-        for (int i = 0; i < C; ++i) {
-            const float yl = __fmul_rn(__fmul_rn(lo[i], r), wl[i]);
-            const float yh = __fmul_rn(__fmul_rn(hi[i], r), wh[i]);
-            const __nv_bfloat16 a = __float2bfloat16_rn(__fsub_rn(__fmul_rn(yl, cv[i]), __fmul_rn(yh, sv[i])));
-            const __nv_bfloat16 b = __float2bfloat16_rn(__fadd_rn(__fmul_rn(yh, cv[i]), __fmul_rn(yl, sv[i])));
-            ol[i] = *reinterpret_cast<const unsigned short*>(&a);
-            oh[i] = *reinterpret_cast<const unsigned short*>(&b);
+        for (int i = 0; i < 8; i += 2) {
+            float a[2], b[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const float yl = __fmul_rn(__fmul_rn(lo[i + k], r), wl[i + k]);
+                const float yh = __fmul_rn(__fmul_rn(hi[i + k], r), wh[i + k]);
+                a[k] = __fsub_rn(__fmul_rn(yl, cv[i + k]), __fmul_rn(yh, sv[i + k]));
+                b[k] = __fadd_rn(__fmul_rn(yh, cv[i + k]), __fmul_rn(yl, sv[i + k]));
+            }
+            ol[i / 2] = pack_bf16x2(a[0], a[1]);
+            oh[i / 2] = pack_bf16x2(b[0], b[1]);
         }
-        *reinterpret_cast<Vec*>(o + lane * C) = *reinterpret_cast<const Vec*>(ol);
-        *reinterpret_cast<Vec*>(o + HALF + lane * C) = *reinterpret_cast<const Vec*>(oh);
+        *reinterpret_cast<uint4*>(o) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+        *reinterpret_cast<uint4*>(o + HALF) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
     }
+}
+
+template <int D>
+const void* qknr_fn()
+{
+    return (const void*)qk_norm_rope_kernel<D, 2>;
 }
 
 }  // namespace
@@ -128,19 +166,21 @@ int launch_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int 
                         const void* k_weight, const float* cos_sin, int max_pos, const long long* positions, float eps,
                         cudaStream_t s)
 {
-    constexpr int kHeadsPerWarp = 4;
-    const long long warps = (long long)T * ((Hq + 2 * Hkv + kHeadsPerWarp - 1) / kHeadsPerWarp);
-    if (warps == 0) return W8_OK;
+    constexpr int kGroupsPerWarp = 2;
+    const int Hn = out == qkv ? Hq + Hkv : Hq + 2 * Hkv;
+    const int hpw = 512 / D;
+    const long long units = (long long)T * ((Hn + hpw - 1) / hpw);
+    if (units == 0) return W8_OK;
+    if (units > 0x7FFFFFFFLL - 256) return W8_ERR_UNSUPPORTED;
+    const long long warps = (units + kGroupsPerWarp - 1) / kGroupsPerWarp;
     const long long blocks = (warps + 3) / 4;
-    if (blocks > 0x7FFFFFFF) return W8_ERR_UNSUPPORTED;
-    const void* fn = D == 64 ? (const void*)qk_norm_rope_kernel<1, kHeadsPerWarp>
-                   : D == 128 ? (const void*)qk_norm_rope_kernel<2, kHeadsPerWarp>
-                              : (const void*)qk_norm_rope_kernel<4, kHeadsPerWarp>;
+    const void* fn = D == 64 ? qknr_fn<64>() : D == 128 ? qknr_fn<128>() : qknr_fn<256>();
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(qkv);
     __nv_bfloat16* op = static_cast<__nv_bfloat16*>(out);
     const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(q_weight);
     const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(k_weight);
-    void* args[] = {(void*)&xp, (void*)&op, (void*)&T, (void*)&Hq, (void*)&Hkv, (void*)&qp, (void*)&kp,
+    int un = (int)units;
+    void* args[] = {(void*)&xp, (void*)&op, (void*)&Hq, (void*)&Hkv, (void*)&Hn, (void*)&un, (void*)&qp, (void*)&kp,
                     (void*)&cos_sin, (void*)&max_pos, (void*)&positions, (void*)&eps};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)blocks);

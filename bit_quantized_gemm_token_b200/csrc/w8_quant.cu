@@ -8,9 +8,11 @@
 //   s = amax / Q (fp32 division; Q = 448 e4m3, 127 int8; s = 1 for an all-zero row),
 //   q = e4m3_rn_satfinite(x / s)  or  clamp(rint(x / s), -127, 127),
 //   UE8M0 scales: the smallest power of two >= amax/448, exponent in [-127, 127].
-// Every division is the IEEE one (__fdiv_rn), never x * (1/s), and no arithmetic is
-// left to compiler contraction (__fmul_rn / __fadd_rn / __fmaf_rn spell out each
-// rounding), so the codes are a deterministic function of the inputs.
+// Every quotient x / s is the correctly rounded IEEE one: silu's division is __fdiv_rn,
+// and the codes take x / s from a row reciprocal with Markstein's correction
+// (w8_codes.cuh, quotient_rn: the same fp32 quotient wherever a code can depend on it).
+// No arithmetic is left to compiler contraction (__fmul_rn / __fadd_rn / __fmaf_rn spell
+// out each rounding), so the codes are a deterministic function of the inputs.
 //
 // Layout of the work: the row kernels give one CTA per row and keep the row in
 // registers (16-byte vector loads, CPT chunks of 8 bf16 per thread); reductions are
@@ -20,6 +22,9 @@
 // the previous grid before it reads or writes anything.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
+
+#include <map>
+#include <mutex>
 
 #include "w8_codes.cuh"
 #include "w8_internal.h"
@@ -45,6 +50,21 @@ __device__ __forceinline__ float block_max(float v, float* red)
     __syncthreads();
     float r = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0f;
     r = warp_max(r);
+    __syncthreads();
+    return r;
+}
+
+// fp64 sum over the CTA (a fixed tree); every thread gets the result.  `red` holds 32.
+__device__ __forceinline__ double block_sum64(double v, double* red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r = __dadd_rn(r, __shfl_xor_sync(0xFFFFFFFFu, r, o));
     __syncthreads();
     return r;
 }
@@ -106,50 +126,74 @@ __device__ __forceinline__ void encode_chunk_grouped(const float (&y)[8], int id
     const float s = scale_from_amax(amax, kE4M3Max, ue8m0);
     if ((idx & 15) == 0) srow[idx >> 4] = s;
     (void)ng;
-    *reinterpret_cast<uint2*>(qrow + (size_t)idx * 8) = encode8<W8_Q_FP8>(y, s);
+    const RowDivisor d = make_divisor(s, amax);
+    *reinterpret_cast<uint2*>(qrow + (size_t)idx * 8) = encode8<W8_Q_FP8>(y, d);
 }
 
 // ------------------------------------------------------------------- per-token rows
+// Rows m = blockIdx.x, + gridDim.x, ...: each CTA issues the loads of its next row before
+// it reduces and encodes the current one, so its loads stay in flight across the row's
+// barriers (the grid is one row per CTA for few rows, the resident CTAs for many).
+template <int CPT>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* xr, int chunks, uint4 (&r)[CPT])
+{
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int idx = threadIdx.x + c * blockDim.x;
+        if (idx < chunks) r[c] = ld_nc_v4(xr + (size_t)idx * 8);
+    }
+}
+
 template <int QFMT, int CPT>
-__global__ void __launch_bounds__(1024) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int K, int ldx,
+__global__ void __launch_bounds__(1024) quant_rows_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, int ldx,
                                                           uint8_t* __restrict__ q, float* __restrict__ scale)
 {
     __shared__ float red[32];
     ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
-    const int m = blockIdx.x;
     const int chunks = K >> 3;
-    const __nv_bfloat16* xr = x + (size_t)m * ldx;
-    uint4 raw[CPT];
-    float amax = 0.0f;
+    uint4 raw[CPT], nxt[CPT];
+    int m = blockIdx.x;
+    load_row<CPT>(x + (size_t)m * ldx, chunks, raw);
+    for (;;) {
+        const int mn = m + (int)gridDim.x;
+        if (mn < M) load_row<CPT>(x + (size_t)mn * ldx, chunks, nxt);
+        float amax = 0.0f;
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-        const int idx = threadIdx.x + c * blockDim.x;
-        if (idx < chunks) {
-            raw[c] = ld_nc_v4(xr + (size_t)idx * 8);
-            float f[8];
-            unpack_bf16x8(raw[c], f);
+        for (int c = 0; c < CPT; ++c) {
+            const int idx = threadIdx.x + c * blockDim.x;
+            if (idx < chunks) {
+                float f[8];
+                unpack_bf16x8(raw[c], f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            }
         }
-    }
-    amax = block_max(amax, red);
-    const float s = scale_from_amax(amax, QFMT == W8_Q_FP8 ? kE4M3Max : kInt8Max, false);
-    if (threadIdx.x == 0) scale[m] = s;
-    uint8_t* qr = q + (size_t)m * K;
+        amax = block_max(amax, red);
+        const float s = scale_from_amax(amax, QFMT == W8_Q_FP8 ? kE4M3Max : kInt8Max, false);
+        if (threadIdx.x == 0) scale[m] = s;
+        const RowDivisor d = make_divisor(s, amax);
+        uint8_t* qr = q + (size_t)m * K;
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) {
-        const int idx = threadIdx.x + c * blockDim.x;
-        if (idx < chunks) {
-            float f[8];
-            unpack_bf16x8(raw[c], f);
-            *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<QFMT>(f, s);
+        for (int c = 0; c < CPT; ++c) {
+            const int idx = threadIdx.x + c * blockDim.x;
+            if (idx < chunks) {
+                float f[8];
+                unpack_bf16x8(raw[c], f);
+                *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<QFMT>(f, d);
+            }
         }
+        if (mn >= M) break;
+        m = mn;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) raw[c] = nxt[c];
     }
 }
 
 // ------------------------------------------------------------------- 1x128 groups
-// A half-warp (16 lanes x 8 elements) per group; scale[m * (K/128) + g].
+// A half-warp (16 lanes x 8 elements) per group; scale[m * (K/128) + g].  (Four groups
+// per half-warp with their loads issued together measured slower on B200: 70 against
+// 64 us for 16384 x 4096.)
 __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16* __restrict__ x, int M, int K,
                                                              int ldx, uint8_t* __restrict__ q,
                                                              float* __restrict__ scale, int ue8m0)
@@ -173,7 +217,8 @@ __global__ void __launch_bounds__(256) quant_group128_kernel(const __nv_bfloat16
     for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(hmask, amax, o));
     const float s = scale_from_amax(amax, kE4M3Max, ue8m0 != 0);
     if (l16 == 0) scale[(size_t)m * gpr + g] = s;
-    *reinterpret_cast<uint2*>(q + (size_t)m * K + (size_t)g * 128 + l16 * 8) = encode8<W8_Q_FP8>(f, s);
+    const RowDivisor d = make_divisor(s, amax);
+    *reinterpret_cast<uint2*>(q + (size_t)m * K + (size_t)g * 128 + l16 * 8) = encode8<W8_Q_FP8>(f, d);
 }
 
 // ------------------------------------------------------------------- 128x128 weight blocks
@@ -204,6 +249,7 @@ __global__ void __launch_bounds__(256) quant_weight_block_kernel(const __nv_bflo
     amax = block_max(amax, red);
     const float s = scale_from_amax(amax, kE4M3Max, ue8m0 != 0);
     if (threadIdx.x == 0) scale[(size_t)bn * nbk + bk] = s;
+    const RowDivisor d = make_divisor(s, amax);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int c = threadIdx.x + i * 256;
@@ -211,7 +257,7 @@ __global__ void __launch_bounds__(256) quant_weight_block_kernel(const __nv_bflo
         if (r < rows && cc < cols) {
             float f[8];
             unpack_bf16x8(raw[i], f);
-            *reinterpret_cast<uint2*>(q + (size_t)(bn * 128 + r) * K + bk * 128 + cc) = encode8<W8_Q_FP8>(f, s);
+            *reinterpret_cast<uint2*>(q + (size_t)(bn * 128 + r) * K + bk * 128 + cc) = encode8<W8_Q_FP8>(f, d);
         }
     }
 }
@@ -220,51 +266,53 @@ __global__ void __launch_bounds__(256) quant_weight_block_kernel(const __nv_bflo
 template <int CPT, bool GROUPED>
 __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16* __restrict__ x,
                                                              const __nv_bfloat16* __restrict__ gamma, float eps,
-                                                             int H, int ldx, uint8_t* __restrict__ q,
+                                                             int M, int H, int ldx, uint8_t* __restrict__ q,
                                                              float* __restrict__ scale, int ue8m0)
 {
     __shared__ DSum redd[32];
+    __shared__ double red64[32];
     __shared__ float red[32];
     ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
     ptx::grid_dep_wait();
+    (void)M;
     const int m = blockIdx.x;
     const int chunks = H >> 3;
-    const __nv_bfloat16* xr = x + (size_t)m * ldx;
     uint4 raw[CPT];
-    DSum ss{0.0, 0.0};
+    load_row<CPT>(x + (size_t)m * ldx, chunks, raw);
+    double ss64 = 0.0;
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
         const int idx = threadIdx.x + c * blockDim.x;
         if (idx < chunks) {
-            raw[c] = ld_nc_v4(xr + (size_t)idx * 8);
             float f[8];
             unpack_bf16x8(raw[c], f);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) ss = dsum_sq(ss, f[i]);
+            for (int i = 0; i < 8; ++i) ss64 = __fma_rn((double)f[i], (double)f[i], ss64);   // squares exact
         }
     }
-    ss = block_sum_dd(ss, redd);
-    // the exact sum of squares rounded once to fp32, then the mean (w8_sumsq.cuh)
-    const float mean = __fdiv_rn(dsum_to_f32(ss), (float)H);
-    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
-    if (GROUPED) {
-        // rms_norm_per_block_quant: y = (x * r) * gamma, then one scale per 1x128 group
-        const int ng = H >> 7;
+    // the exact sum of squares rounded once to fp32 (w8_sumsq.cuh): the fp64 sum when its
+    // error bound settles the rounding (no term meets more than H roundings), else the
+    // double-double sum; the CTA-wide sum is the same in every thread, so is the branch
+    ss64 = block_sum64(ss64, red64);
+    float ssf;
+    if (!sq_round_certain(ss64, H, &ssf)) {
+        DSum ss{0.0, 0.0};
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
             const int idx = threadIdx.x + c * blockDim.x;
             if (idx < chunks) {
-                float f[8], g[8], y[8];
+                float f[8];
                 unpack_bf16x8(raw[c], f);
-                unpack_bf16x8(ld_nc_v4(gamma + (size_t)idx * 8), g);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(f[i], r), g[i]);
-                encode_chunk_grouped(y, idx, ng, ue8m0 != 0, q + (size_t)m * H, scale + (size_t)m * ng);
+                for (int i = 0; i < 8; ++i) ss = dsum_sq(ss, f[i]);
             }
         }
-        return;
+        ssf = dsum_to_f32(block_sum_dd(ss, redd));
     }
-    // y = (x * r) * gamma, recomputed in the second pass rather than kept
+    const float mean = __fdiv_rn(ssf, (float)H);
+    const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(mean, eps)));
+    // y = (x * r) * gamma, kept in registers for the codes
+    float y[CPT][8];
     float amax = 0.0f;
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
@@ -274,40 +322,40 @@ __global__ void __launch_bounds__(1024) rmsnorm_quant_kernel(const __nv_bfloat16
             unpack_bf16x8(raw[c], f);
             unpack_bf16x8(ld_nc_v4(gamma + (size_t)idx * 8), g);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(f[i], r), g[i])));
+            for (int i = 0; i < 8; ++i) {
+                y[c][i] = __fmul_rn(__fmul_rn(f[i], r), g[i]);
+                amax = fmaxf(amax, fabsf(y[c][i]));
+            }
         }
+    }
+    if (GROUPED) {
+        // rms_norm_per_block_quant: one scale per 1x128 group of y
+        const int ng = H >> 7;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int idx = threadIdx.x + c * blockDim.x;
+            if (idx < chunks) encode_chunk_grouped(y[c], idx, ng, ue8m0 != 0, q + (size_t)m * H, scale + (size_t)m * ng);
+        }
+        return;
     }
     amax = block_max(amax, red);
     const float s = scale_from_amax(amax, kE4M3Max, false);
     if (threadIdx.x == 0) scale[m] = s;
+    const RowDivisor d = make_divisor(s, amax);
     uint8_t* qr = q + (size_t)m * H;
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
         const int idx = threadIdx.x + c * blockDim.x;
-        if (idx < chunks) {
-            float f[8], g[8], y[8];
-            unpack_bf16x8(raw[c], f);
-            unpack_bf16x8(ld_nc_v4(gamma + (size_t)idx * 8), g);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(__fmul_rn(f[i], r), g[i]);
-            *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<W8_Q_FP8>(y, s);
-        }
+        if (idx < chunks) *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<W8_Q_FP8>(y[c], d);
     }
 }
 
 // ------------------------------------------------------------------- silu_and_mul + quant
 template <int CPT, bool GROUPED>
-__global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat16* __restrict__ xgu, int I, int ld,
-                                                              uint8_t* __restrict__ q, float* __restrict__ scale,
-                                                              int ue8m0)
+__device__ __forceinline__ void silu_row(const uint4 (&rg)[CPT], const uint4 (&ru)[CPT], int m, int I, uint8_t* q,
+                                         float* scale, int ue8m0, float* red)
 {
-    __shared__ float red[32];
-    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
-    ptx::grid_dep_wait();
-    const int m = blockIdx.x;
     const int chunks = I >> 3;
-    const __nv_bfloat16* gr = xgu + (size_t)m * ld;
-    const __nv_bfloat16* ur = gr + I;
     float h[CPT][8];
     float amax = 0.0f;
 #pragma unroll
@@ -315,8 +363,8 @@ __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat1
         const int idx = threadIdx.x + c * blockDim.x;
         if (idx < chunks) {
             float g[8], u[8];
-            unpack_bf16x8(ld_nc_v4(gr + (size_t)idx * 8), g);
-            unpack_bf16x8(ld_nc_v4(ur + (size_t)idx * 8), u);
+            unpack_bf16x8(rg[c], g);
+            unpack_bf16x8(ru[c], u);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float den = __fadd_rn(1.0f, exp_cw(-g[i]));
@@ -338,26 +386,55 @@ __global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat1
     amax = block_max(amax, red);
     const float s = scale_from_amax(amax, kE4M3Max, false);
     if (threadIdx.x == 0) scale[m] = s;
+    const RowDivisor d = make_divisor(s, amax);
     uint8_t* qr = q + (size_t)m * I;
 #pragma unroll
     for (int c = 0; c < CPT; ++c) {
         const int idx = threadIdx.x + c * blockDim.x;
-        if (idx < chunks) *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<W8_Q_FP8>(h[c], s);
+        if (idx < chunks) *reinterpret_cast<uint2*>(qr + (size_t)idx * 8) = encode8<W8_Q_FP8>(h[c], d);
     }
 }
 
-// Threads per row and chunks per thread for a row of `chunks` 16-byte chunks: the
-// fewest chunks per thread (1, 2 or 4) that fits in 1024 threads.
-inline bool row_shape(int chunks, int* threads, int* cpt)
+template <int CPT, bool GROUPED>
+__global__ void __launch_bounds__(1024) silu_mul_quant_kernel(const __nv_bfloat16* __restrict__ xgu, int M, int I,
+                                                              int ld, uint8_t* __restrict__ q,
+                                                              float* __restrict__ scale, int ue8m0)
 {
-    for (int c : {1, 2, 4}) {
+    __shared__ float red[32];
+    ptx::grid_dep_launch();   // dependents may launch now; they wait for this grid themselves
+    ptx::grid_dep_wait();
+    (void)M;
+    const int m = blockIdx.x;
+    const int chunks = I >> 3;
+    uint4 rg[CPT], ru[CPT];
+    load_row<CPT>(xgu + (size_t)m * ld, chunks, rg);
+    load_row<CPT>(xgu + (size_t)m * ld + I, chunks, ru);
+    silu_row<CPT, GROUPED>(rg, ru, m, I, q, scale, ue8m0, red);
+}
+
+// Threads per row and chunks per thread for `rows` rows of `chunks` 16-byte chunks.  Each
+// thread issues all its loads before the row's reductions.  Few rows (decode) are bound by
+// the latency of one CTA's chain of loads, reductions and stores: the fewest chunks per
+// thread (1, 2 or 4) that fits in 1024 threads keeps that chain short.  Many rows are
+// bound by HBM: the most chunks per thread (4, 2 or 1) that still leaves 64 threads puts
+// more bytes in flight per SM, whose thread slots run out before its CTA slots (16384
+// rows of 4096 bf16: 63 -> 51 us on B200, while 32 rows lose ~4 us to the longer chain).
+constexpr int kManyRows = 1024;
+
+inline bool row_shape(int rows, int chunks, int* threads, int* cpt, int many_max = 4)
+{
+    static const int few[3] = {1, 2, 4}, many[3] = {4, 2, 1};
+    const int* order = rows >= kManyRows ? many : few;
+    for (int i = 0; i < 3; ++i) {
+        const int c = order[i];
         const int t = (chunks + c - 1) / c;
-        if (t <= 1024) {
-            *cpt = c;
-            *threads = ((t + 31) / 32) * 32;
-            if (*threads < 64) *threads = 64;
-            return true;
-        }
+        if (t > 1024) continue;
+        if (rows >= kManyRows && ((t < 64 && c > 1) || (c > many_max && (chunks + many_max - 1) / many_max <= 1024)))
+            continue;
+        *cpt = c;
+        *threads = ((t + 31) / 32) * 32;
+        if (*threads < 64) *threads = 64;
+        return true;
     }
     return false;
 }
@@ -379,15 +456,40 @@ cudaError_t launch(const void* fn, dim3 grid, dim3 block, void** args, cudaStrea
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? W8_OK : W8_ERR_CUDA; }
 
+// Grid of a row kernel: one CTA per row for few rows; for many rows, the CTAs that fit on
+// the GPU at once (occupancy of this kernel at this block size, cached), each looping over
+// rows.
+unsigned row_grid(const void* fn, int threads, int M)
+{
+    if (M < kManyRows) return (unsigned)M;
+    int sms = 0;
+    if (check_device(&sms) != W8_OK || sms <= 0) return (unsigned)M;
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, int> cache;
+    int per = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = cache.find({fn, threads});
+        if (it != cache.end()) per = it->second;
+    }
+    if (per == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, threads, 0) != cudaSuccess || per < 1) per = 1;
+        std::lock_guard<std::mutex> lk(mu);
+        cache[{fn, threads}] = per;
+    }
+    const long long g = (long long)sms * per;
+    return (unsigned)(g < M ? g : M);
+}
+
 }  // namespace
 
 int launch_quant_rows(int qfmt, const void* x, int M, int K, int ldx, void* q, float* scale, cudaStream_t s)
 {
     int threads, cpt;
-    if (!row_shape(K / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
+    if (!row_shape(M, K / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
     uint8_t* qp = static_cast<uint8_t*>(q);
-    void* args[] = {(void*)&xp, (void*)&K, (void*)&ldx, (void*)&qp, (void*)&scale};
+    void* args[] = {(void*)&xp, (void*)&M, (void*)&K, (void*)&ldx, (void*)&qp, (void*)&scale};
     const void* fn = nullptr;
     if (qfmt == W8_Q_FP8)
         fn = cpt == 1 ? (const void*)quant_rows_kernel<W8_Q_FP8, 1>
@@ -396,7 +498,7 @@ int launch_quant_rows(int qfmt, const void* x, int M, int K, int ldx, void* q, f
         fn = cpt == 1 ? (const void*)quant_rows_kernel<W8_Q_INT8, 1>
                       : cpt == 2 ? (const void*)quant_rows_kernel<W8_Q_INT8, 2>
                                  : (const void*)quant_rows_kernel<W8_Q_INT8, 4>;
-    return status_of(launch(fn, dim3(M), dim3(threads), args, s));
+    return status_of(launch(fn, dim3(row_grid(fn, threads, M)), dim3(threads), args, s));
 }
 
 int launch_quant_group128(const void* x, int M, int K, int ldx, void* q, float* scale, int ue8m0, cudaStream_t s)
@@ -424,11 +526,12 @@ int launch_rmsnorm_quant(const void* x, const void* gamma, float eps, int M, int
                          int group, int ue8m0, cudaStream_t s)
 {
     int threads, cpt;
-    if (!row_shape(H / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
+    if (!row_shape(M, H / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
     const __nv_bfloat16* gp = static_cast<const __nv_bfloat16*>(gamma);
     uint8_t* qp = static_cast<uint8_t*>(q);
-    void* args[] = {(void*)&xp, (void*)&gp, (void*)&eps, (void*)&H, (void*)&ldx, (void*)&qp, (void*)&scale, (void*)&ue8m0};
+    void* args[] = {(void*)&xp, (void*)&gp, (void*)&eps, (void*)&M, (void*)&H, (void*)&ldx, (void*)&qp, (void*)&scale,
+                    (void*)&ue8m0};
     const void* fn;
     if (group)
         fn = cpt == 1 ? (const void*)rmsnorm_quant_kernel<1, true>
@@ -443,10 +546,10 @@ int launch_silu_mul_quant(const void* xgu, int M, int I, int ld, void* q, float*
                           cudaStream_t s)
 {
     int threads, cpt;
-    if (!row_shape(I / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
+    if (!row_shape(M, I / 8, &threads, &cpt)) return W8_ERR_UNSUPPORTED;
     const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(xgu);
     uint8_t* qp = static_cast<uint8_t*>(q);
-    void* args[] = {(void*)&xp, (void*)&I, (void*)&ld, (void*)&qp, (void*)&scale, (void*)&ue8m0};
+    void* args[] = {(void*)&xp, (void*)&M, (void*)&I, (void*)&ld, (void*)&qp, (void*)&scale, (void*)&ue8m0};
     const void* fn;
     if (group)
         fn = cpt == 1 ? (const void*)silu_mul_quant_kernel<1, true>

@@ -4,12 +4,13 @@
 // "Patron de fusion del forward pass": rms_norm fused with the fp8 quant) is the exact
 // sum of the squared bf16 values, rounded to fp32 (nearest, ties to even), so that the
 // result does not depend on the order in which threads add.  Each square of a bf16 is
-// exact in fp64; the squares are added as double-doubles (hi + lo, Knuth's TwoSum for
-// every addition of a term or of a partial sum), which carries about 106 significant
-// bits, and hi + lo is rounded once to fp32 by locating it between its two fp32
-// neighbours.  The result is the correctly rounded fp32 of the exact sum unless that
-// sum lies within about 2^-85 (relative) of an fp32 rounding midpoint without being on
-// it -- which no sum of a few thousand bf16 squares of ordinary range does.
+// exact in fp64.  A plain fp64 sum in any order, with its error bound, almost always
+// settles the fp32 rounding (sq_round_certain below).  Otherwise the squares are added
+// as double-doubles (hi + lo, Knuth's TwoSum for every
+// addition of a term or of a partial sum), which carries about 106 significant bits, and
+// hi + lo is rounded once to fp32 by locating it between its two fp32 neighbours: the
+// correctly rounded fp32 of the exact sum unless that sum lies within about 2^-85
+// (relative) of an fp32 rounding midpoint without being on it.
 #pragma once
 #include <cstdint>
 
@@ -45,6 +46,31 @@ __device__ __forceinline__ DSum dsum_sq(DSum s, float x)
 __device__ __forceinline__ DSum dsum_shfl_xor(DSum s, int o)
 {
     return DSum{__shfl_xor_sync(0xFFFFFFFFu, s.hi, o), __shfl_xor_sync(0xFFFFFFFFu, s.lo, o)};
+}
+
+// Rounding certificate of a plain fp64 sum of squares.  The fp64 sum s of nonnegative
+// terms (each square of a bf16 is exact in fp64) added in any order in which no term
+// passes through more than d roundings differs from the exact sum S by at most
+// gamma_d S, gamma_d = d u / (1 - d u), u = 2^-53 (the standard bound for recursive and
+// pairwise summation; any order of n terms has d <= n - 1).  With d u <= 1/4 that puts S
+// in [s - e, s + e], e = d 2^-52 s.  RN to fp32 is monotone, so when both ends of the
+// interval (rounded outward in fp64) round to the same fp32, S rounds to it as well:
+// that value is the correctly rounded exact sum, whatever the order of the fp64
+// additions.  A non-finite s is already the answer: squares of finite bf16 values (below
+// 2^256) cannot overflow an fp64 sum, so s = +inf means an infinite input (the exact sum
+// is +inf) and NaN a NaN input.  The test fails only for an S within about d 2^-52
+// (relative) of an fp32 rounding midpoint; the caller then recomputes with double-doubles.
+__device__ __forceinline__ bool sq_round_certain(double s, int depth, float* out)
+{
+    const double e = __dmul_ru(s, (double)depth * 0x1p-52);
+    const float lo = __double2float_rn(__dsub_rd(s, e));
+    const float hi = __double2float_rn(__dadd_ru(s, e));
+    if (!isfinite(s)) {
+        *out = __double2float_rn(s);
+        return true;
+    }
+    *out = lo;
+    return lo == hi;
 }
 
 // hi + lo rounded once to fp32, to nearest, ties to even

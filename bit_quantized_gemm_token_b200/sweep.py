@@ -92,6 +92,20 @@ def candidates(fmt, M, N, K, quick=False, families=("swap", "bm64", "decode")):
         v = shipped_variant(fmt, M, N, K)
         if v:
             out.append(v)
+    if "mid" in families:
+        # token counts past the decode form: 256 x 256 tiles on CTA pairs, and the one-CTA
+        # Standard loops with 128 x 128 / 128 x 256 tiles whole, split over K or balanced
+        for stages in (0, 4, 6):
+            out.append(w8.variant(False, 1, 256, stages=stages, pair=True))
+        for split in (2, 4, 8):
+            for stages in (0, 4):
+                out.append(w8.variant(False, split, 256, stages=stages, pair=True))
+        for bn in (128, 256):
+            for kind, arg in [("split", 1), ("split", 2), ("split", 4), ("split", 8), ("stream", 1), ("stream", 2)]:
+                if kind == "stream":
+                    out.append(w8.variant(False, 1, bn, stream=True, cps=arg))
+                else:
+                    out.append(w8.variant(False, arg, bn))
     if "swap" not in families:
         return _legal(fmt, M, N, K, out)
     bns = [b for b in (16, 32, 64) if b >= min(M, 64)][:2]
@@ -253,10 +267,13 @@ def main():
     ap.add_argument("--quick", action="store_true", help="default pipeline depths only")
     ap.add_argument("--formats", default="0,1,2")
     ap.add_argument("--families", default="swap,bm64,decode",
-                    help="candidate families: swap (Swap-AB), bm64 (64-row token tile), decode, shipped (the "
-                         "current table's entry)")
+                    help="candidate families: swap (Swap-AB), bm64 (64-row token tile), decode, mid (CTA pairs "
+                         "and one-CTA Standard loops for larger token counts), shipped (the current table's "
+                         "entry)")
     ap.add_argument("--log", default="")
+    ap.add_argument("--ms", default=",".join(str(m) for m in MS), help="token counts to sweep")
     args = ap.parse_args()
+    ms = [int(m) for m in args.ms.split(",")]
     families = tuple(args.families.split(","))
     # rows of formats not swept now are kept from the table being replaced
     kept = []
@@ -266,7 +283,7 @@ def main():
     if os.path.exists(args.out):
         for line in open(args.out):
             f = line.split("#")[0].split()
-            if len(f) == 5 and int(f[0]) not in fmts_swept:
+            if len(f) == 5 and (int(f[0]) not in fmts_swept or int(f[3]) not in ms):
                 kept.append((int(f[0]), int(f[1]), int(f[2]), int(f[3]), int(f[4], 16)))
     os.environ["W8_TABLE"] = "none"
     w8.w8_clear_table()
@@ -279,8 +296,8 @@ def main():
     top_n = 8
     for fmt in fmts:
         shapes = BLOCK if fmt >= 2 else DENSE
-        probs = [Problem(fmt, N, K, MS, dev) for (K, N) in shapes]
-        for M in MS:
+        probs = [Problem(fmt, N, K, ms, dev) for (K, N) in shapes]
+        for M in ms:
             ref_v = default_variant(fmt, M)
             cands = []
             for prob in probs:

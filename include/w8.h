@@ -116,16 +116,21 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 block, so split_k must not exceed ceil(K / (128 * kps)).
  *   ctas/SM       bits 22..23, CTAs per SM for W8_V_STREAM and the Standard loop
  *                 (0 = 1).
- *   W8_V_PAIR     Standard full-K tile loop (tile 256, split = 0, no W8_V_STREAM /
- *                 W8_V_CLUSTER / W8_V_BM64; FP8-dynamic or INT8) over 256-token x
- *                 256-weight-row tiles, each computed by a cluster of two CTAs on two SMs
- *                 with one 256-row tensor-core MMA (cta_group::2).  Each CTA loads 128
- *                 token rows and 128 weight rows per K block, and its tensor memory holds
- *                 its 128 output rows; the pairs take whole tiles in contiguous runs.
- *                 Stages default to 5.  The same sum as the one-CTA Standard loop: one
- *                 accumulator over the whole K range, K blocks in order (INT8
- *                 accumulators are exact).  For prefill sizes; with PDL the kernel waits
- *                 for the kernels ahead before its first load.
+ *   W8_V_PAIR     Standard tile loop (tile 256, no W8_V_STREAM / W8_V_CLUSTER /
+ *                 W8_V_BM64; FP8-dynamic or INT8) over 256-token x 256-weight-row tiles,
+ *                 each computed by a cluster of two CTAs on two SMs with one 256-row
+ *                 tensor-core MMA (cta_group::2).  Each CTA loads 128 token rows and 128
+ *                 weight rows per K block, and its tensor memory holds its 128 output
+ *                 rows.  split field 0: the pairs take whole tiles in contiguous runs, one
+ *                 accumulator over the whole K range, K blocks in order (the one-CTA
+ *                 Standard loop's sum), no workspace.  split = 2, 4 or 8: one (tile, K
+ *                 chunk) unit per pair -- legal only while tiles x split <= SMs / 2 and
+ *                 split <= ceil(K / 128) -- each CTA's partial sums go to a workspace
+ *                 slot and the last contributor of each half-tile adds the split
+ *                 partials in chunk order (a fixed order), scales and stores; workspace
+ *                 as for the split partitions (256 KiB of counters, then 256 KiB per
+ *                 unit).  Stages default to 5.  INT8 accumulators are exact either way.
+ *                 With PDL the kernel waits for the kernels ahead before its first load.
  *   W8_V_DECODE   decode form (M <= 64; FP8-dynamic or INT8; no W8_V_SWAP_AB / W8_V_STREAM /
  *                 W8_V_CLUSTER / W8_V_BM64 / W8_V_PAIR): the tokens occupy the tensor
  *                 core's 64-row operand and BN = 16 * (tile + 1) weight rows (64..256) its
@@ -303,8 +308,8 @@ W8_API size_t w8_grouped_gemm_workspace_size(int fmt, int E, int T, int N, int K
  *   positions int64 [T] in [0, max_pos): a position outside records W8_ERR_INVALID_ARG
  *             in the device status word (w8_device_status) and leaves that token's
  *             query and key heads unwritten.
- * D must be 64, 128 or 256 (W8_ERR_UNSUPPORTED otherwise); qkv, out and the weights
- * 8-byte aligned, cos_sin 4-byte, positions 8-byte (W8_ERR_ALIGNMENT otherwise). */
+ * D must be 64, 128 or 256 (W8_ERR_UNSUPPORTED otherwise); qkv, out, the weights and
+ * cos_sin 16-byte aligned, positions 8-byte (W8_ERR_ALIGNMENT otherwise). */
 W8_API int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, int D, const void* q_weight,
                            const void* k_weight, const float* cos_sin, int max_pos, const int64_t* positions,
                            float eps, w8_stream_t stream);
@@ -366,6 +371,37 @@ W8_API int w8_linear_debug(int fmt, const void* x, int ldx, const void* W_q, con
  * stream are fine.  Errors: as w8_gemm. */
 W8_API int w8_gemm_noalloc(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                            void* out, int M, int N, int K, int variant, w8_stream_t stream);
+
+/* Failure-path check of the bounded device waits: runs the decode-form GEMM `variant`
+ * resolves to (W8_ERR_UNSUPPORTED for other forms) with its producer issuing no loads,
+ * so that the tensor core never gets operands, and with every wait bounded by wait_us
+ * microseconds (1 .. 1e6) instead of the normal second.  Nothing is ever in flight: the
+ * MMA warp's wait for the first stage runs out, the kernel records W8_ERR_DEVICE_TIMEOUT
+ * in the device status word (w8_device_status), releases its tensor memory and returns
+ * without writing `out`.  The arguments are w8_gemm's (no workspace: the decode form
+ * needs none).  Returns the launch status; the timeout shows in w8_device_status once
+ * the work has completed.  For testing that a wait which cannot end leaves the GPU and
+ * the context usable. */
+W8_API int w8_gemm_timeout_debug(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
+                                 void* out, int M, int N, int K, int variant, int wait_us, w8_stream_t stream);
+
+/* Self-check of the quantizers' division-free quotient (every code of w8_quant_per_token,
+ * w8_rmsnorm_quant, w8_silu_mul_quant and the fused form of w8_linear is formed from
+ * x / s computed with a row reciprocal and Markstein's correction) against the IEEE
+ * quotient x / s that defines the codes.  Scale rule: mode % 3 = 0: amax / 448 with e4m3
+ * codes, 1: amax / 127 with int8 codes, 2: UE8M0 scales with e4m3 codes.  Modes 0..2
+ * enumerate every bf16 amax (smallest subnormal to +inf) and every bf16 x with |x| <= amax,
+ * both signs (about 1.1e9 pairs each); modes 3..5 take 2^30 fp32 pairs from a
+ * counter-based hash (random finite amax; x random with |x| <= amax, or within 3 ulps of a
+ * code's rounding midpoint times s).  A pair fails when the two codes differ, or when the
+ * IEEE quotient is at least 2^-10 in magnitude (where a code can depend on it) and the
+ * two quotients differ in any bit.  Adds the number
+ * of failing pairs to *mismatches; first_bad[0..1] receive (amax bits | 0x80000000, x bits)
+ * of one failing pair if first_bad[0] is 0 (bf16 modes: the bf16 patterns in the high
+ * halves).  Both are device memory owned by the caller (zero them first); asynchronous on
+ * `stream`.  Errors: INVALID_ARG (mode outside 0..5, null pointers), NO_DEVICE, CUDA. */
+W8_API int w8_selfcheck_quotient(int mode, unsigned long long* mismatches, unsigned int* first_bad,
+                                 w8_stream_t stream);
 
 /* CTAs of the kernel `variant` (AUTO resolved) selects for this shape that can be resident
  * on one SM together, from its registers, shared memory and threads (the CUDA occupancy

@@ -73,6 +73,8 @@ def test_bad_arguments_rejected_before_device(L):
         w8.W8_ERR_UNSUPPORTED
     assert L.w8_qk_norm_rope(ctypes.c_void_p((1 << 20) + 2), p16, 1, 2, 1, 128, p16, p16, p16, 8, p16,
                              ctypes.c_float(1e-6), NULL) == w8.W8_ERR_ALIGNMENT
+    assert L.w8_qk_norm_rope(p16, p16, 1, 2, 1, 128, p16, p16, ctypes.c_void_p((1 << 20) + 8), 8, p16,
+                             ctypes.c_float(1e-6), NULL) == w8.W8_ERR_ALIGNMENT   # cos/sin table 16-byte
     assert L.w8_qk_norm_rope(NULL, p16, 1, 2, 1, 128, p16, p16, p16, 8, p16, ctypes.c_float(1e-6), NULL) == \
         w8.W8_ERR_INVALID_ARG
 

@@ -143,6 +143,40 @@ def test_pair_tiles(orc, fmt, M, N, K):
     assert w8.w8_device_status(clear=True) == 0
 
 
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(300, 600, 2048), (256, 512, 1040), (64, 300, 4096), (513, 256, 1024)])
+def test_pair_split_k(orc, fmt, M, N, K):
+    """CTA-pair tiles with a K split (one (tile, K chunk) unit per pair, the last
+    contributor adding the chunks in order): ragged token, weight and K tiles, split up
+    to one K block per chunk; the oracle's outputs within the GEMM bound, INT8 int32
+    accumulators exactly, and the same bytes on a second call with the same workspace."""
+    Aq, sA, Wq, sW, ref, acc = operands(orc, fmt, M, N, K)
+    A, SA, W, SW = dev_codes(Aq, fmt), dev_f32(sA), dev_codes(Wq, fmt), dev_f32(sW)
+    tiles = -(-M // 256) * -(-N // 256)
+    kbs = -(-K // 128)
+    ws = w8.Workspace()
+    ran = 0
+    for S in (2, 4, 8):
+        if tiles * S > 74 or S > kbs:
+            with pytest.raises(w8.W8Error):
+                w8.w8_gemm_resolve_variant(fmt, M, N, K, w8.variant(False, S, 256, pair=True))
+            continue
+        for v in (w8.variant(False, S, 256, pair=True), w8.variant(False, S, 256, pair=True, pdl=True, stages=3)):
+            o1 = w8.w8_gemm(fmt, A, SA, W, SW, variant=v, workspace=ws).clone()
+            o2 = w8.w8_gemm(fmt, A, SA, W, SW, variant=v, workspace=ws).clone()
+            torch.cuda.synchronize()
+            assert_bf16_close(o1, ref, "pair split %d %s" % (S, (M, N, K)))
+            assert torch.equal(o1, o2)
+            if fmt == 1:
+                a32 = w8.w8_gemm_i32_debug(A, W, variant=v, workspace=ws)
+                torch.cuda.synchronize()
+                assert np.array_equal(a32.cpu().numpy().astype(np.int64), acc)
+            ran += 1
+    assert ran > 0
+    assert int(ws.buf[:256 * 1024].sum()) == 0      # counter area back to zero
+    assert w8.w8_device_status(clear=True) == 0
+
+
 def test_repeated_calls_reuse_workspace(orc):
     """Counters are left at zero: the same workspace serves back-to-back split calls,
     and the results are bit-identical run to run (fixed reduction order)."""

@@ -68,3 +68,29 @@ def test_bad_sizes_rejected():
         w8.w8_qk_norm_rope(x, 2, 1, 96, w, w, torch.zeros((4, 96), device="cuda"),
                            torch.zeros(2, dtype=torch.int64, device="cuda"))
     assert e.value.code == w8.W8_ERR_UNSUPPORTED
+
+
+def test_heads_on_fp32_midpoints(orc):
+    """Heads whose exact sum of squares lies on or a hair past an fp32 rounding midpoint
+    (1 + 2^-24) sit beside ordinary heads in the same warp: the heads whose fp64 sum
+    cannot settle the rounding recompute it with double-doubles while their neighbours
+    do not, and every output still equals the oracle's."""
+    T, Hq, Hkv, D = 6, 8, 2, 128
+    qkv, qw, kw, pos, table = case(T, Hq, Hkv, D, seed=77)
+    x = qkv.float().view(T, Hq + 2 * Hkv, D)
+    for t in range(T):
+        for h in range(t % 3, Hq + Hkv, 3):
+            x[t, h] = 0.0
+            x[t, h, 0] = 1.0
+            x[t, h, 5] = 2.0 ** -12
+            if (t + h) % 2:
+                x[t, h, D - 1] = 2.0 ** -50
+    qkv = x.view(T, -1).to(torch.bfloat16)
+    want = oracle_out(orc, qkv, qw, kw, pos, table, Hq, Hkv, D)
+    for inplace in (False, True):
+        xd = qkv.cuda()
+        got = w8.w8_qk_norm_rope(xd, Hq, Hkv, D, qw.cuda(), kw.cuda(), table.cuda(), pos.cuda(),
+                                 out=xd if inplace else None)
+        torch.cuda.synchronize()
+        assert np.array_equal(synth.bf16_bits(got.cpu()), want), inplace
+    assert w8.w8_device_status(clear=True) == 0

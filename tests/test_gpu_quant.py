@@ -147,3 +147,24 @@ def test_rmsnorm_sum_of_squares_at_fp32_midpoints(orc):
         naive = np.float32(np.sum(xf[i] * xf[i]))
         r = np.float32(1.0) / np.sqrt(naive / np.float32(H))
         assert np.float32(r / np.float32(448.0)) != os_[i]
+
+
+def test_rmsnorm_quant_independent_of_element_order(orc):
+    """Permuting a row's elements (and gamma with them) permutes the codes and leaves the
+    scale alone: the sum of squares is the exact sum rounded once, so the order in which
+    the GPU's threads add cannot show.  Rows with a wide spread of magnitudes (a few
+    values 2^20 times the rest) make a plain fp32 sum order-dependent."""
+    M, H = 16, 4096
+    x = synth.activations(M, H, seed=4400).float()
+    x[:, ::512] *= 2.0 ** 20
+    x = x.to(torch.bfloat16)
+    g = synth.gamma(H, seed=4401)
+    perm = torch.from_numpy(np.random.default_rng(4402).permutation(H))
+    q, s = w8.w8_rmsnorm_quant(x.cuda(), g.cuda(), 1e-6)
+    qp, sp = w8.w8_rmsnorm_quant(x[:, perm].contiguous().cuda(), g[perm].contiguous().cuda(), 1e-6)
+    torch.cuda.synchronize()
+    assert torch.equal(s.cpu(), sp.cpu())
+    assert np.array_equal(u8(q)[:, perm.numpy()], u8(qp))
+    oq, os_ = orc.rmsnorm_quant(bits(x), bits(g), 1e-6)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(u8(q), oq)
