@@ -551,46 +551,62 @@ def time_extras(dev, peak):
     res["block_fp8_decode"] = format_chain(dev, g, w8, w8.W8_FMT_BLOCK_FP8,
                                            [(5120, 10240), (5120, 51200), (25600, 5120), (4096, 6144)], [1, 8, 32], peak)
     res["mlp_chain"] = mlp_chain(dev, g, w8, peak, fp8_peak)
+    res["mlp_chain_block_fp8"] = mlp_chain(dev, g, w8, peak, fp8_peak, fmt=w8.W8_FMT_BLOCK_FP8)
     return res
 
 
-def mlp_chain(dev, g, w8, peak, fp8_peak):
-    """The MLP block hidden 4096 / intermediate 12288 in FP8-dynamic: rms_norm + quant,
-    gate_up GEMM, silu_and_mul + quant, down GEMM (AUTO + PDL, one CUDA graph per token
-    count, two weight copies in rotation).  Decode token counts in TB/s of algorithmic
-    bytes, prefill ones in TFLOP/s of the two GEMMs."""
+def mlp_chain(dev, g, w8, peak, fp8_peak, fmt=0):
+    """The MLP block hidden 4096 / intermediate 12288: rms_norm + quant, gate_up GEMM,
+    silu_and_mul + quant, down GEMM (AUTO + PDL, one CUDA graph per token count, two
+    weight copies in rotation), in FP8-dynamic (per-token scales, per-channel weights) or
+    Block-FP8 (fmt 2: 1 x 128 activation groups, 128 x 128 weight blocks).  Decode token
+    counts in TB/s of algorithmic bytes, prefill ones in TFLOP/s of the two GEMMs."""
     import torch
     H, I = 4096, 12288
+    block = fmt >= 2
     gamma = (torch.rand(H, device=dev, generator=g) + 0.5).to(torch.bfloat16)
+    wq = (lambda wb: w8.w8_quant_weight_block(wb)) if block else (lambda wb: w8.w8_quant_per_token(wb))
     Wgu, Wd = [], []
     for _ in range(2):
-        Wgu.append(w8.w8_quant_per_token((torch.randn(2 * I, H, device=dev, generator=g) * 0.02).to(torch.bfloat16)))
-        Wd.append(w8.w8_quant_per_token((torch.randn(H, I, device=dev, generator=g) * 0.02).to(torch.bfloat16)))
+        Wgu.append(wq((torch.randn(2 * I, H, device=dev, generator=g) * 0.02).to(torch.bfloat16)))
+        Wd.append(wq((torch.randn(H, I, device=dev, generator=g) * 0.02).to(torch.bfloat16)))
     ws = w8.Workspace(dev)
     v = w8.W8_VARIANT_AUTO | w8.W8_V_PDL
     out = {}
-    for M in (1, 8, 32, 256, 1024, 4096):
+    for M in ((1, 8, 32, 256, 1024) if block else (1, 8, 32, 256, 1024, 4096)):
         x = torch.randn(M, H, device=dev, generator=g).to(torch.bfloat16)
         q1 = torch.empty(M, H, dtype=torch.float8_e4m3fn, device=dev)
-        s1 = torch.empty(M, device=dev)
+        s1 = torch.empty(M, H // 128, device=dev) if block else torch.empty(M, device=dev)
         gu = torch.empty(M, 2 * I, dtype=torch.bfloat16, device=dev)
         q2 = torch.empty(M, I, dtype=torch.float8_e4m3fn, device=dev)
-        s2 = torch.empty(M, device=dev)
+        s2 = torch.empty(M, I // 128, device=dev) if block else torch.empty(M, device=dev)
         y = torch.empty(M, H, dtype=torch.bfloat16, device=dev)
         reps = 4 if M <= 32 else 2
 
         def chain():
             for r in range(reps):
-                w8.w8_rmsnorm_quant(x, gamma, 1e-6, q=q1, scale=s1)
-                w8.w8_gemm(0, q1, s1, Wgu[r % 2][0], Wgu[r % 2][1], out=gu, variant=v, workspace=ws)
-                w8.w8_silu_mul_quant(gu, q=q2, scale=s2)
-                w8.w8_gemm(0, q2, s2, Wd[r % 2][0], Wd[r % 2][1], out=y, variant=v, workspace=ws)
+                if block:
+                    w8.w8_rmsnorm_quant_group(x, gamma, 1e-6, q=q1, scale=s1)
+                else:
+                    w8.w8_rmsnorm_quant(x, gamma, 1e-6, q=q1, scale=s1)
+                w8.w8_gemm(fmt, q1, s1, Wgu[r % 2][0], Wgu[r % 2][1], out=gu, variant=v, workspace=ws)
+                if block:
+                    w8.w8_silu_mul_quant_group(gu, q=q2, scale=s2)
+                else:
+                    w8.w8_silu_mul_quant(gu, q=q2, scale=s2)
+                w8.w8_gemm(fmt, q2, s2, Wd[r % 2][0], Wd[r % 2][1], out=y, variant=v, workspace=ws)
             return 4 * reps
         ms, _ = time_graph(chain, 5, 3, 1)
         us = ms * 1e3 / reps
         if M <= 32:
-            byts = (2 * M * H + 2 * H + M * H + 4 * M) + gemm_bytes(M, 2 * I, H) \
-                + (2 * M * 2 * I + M * I + 4 * M) + gemm_bytes(M, H, I)
+            if block:   # group scales of the activations, 128 x 128 block scales of the weights
+                byts = (2 * M * H + 2 * H + M * H + 4 * M * H // 128) \
+                    + (2 * I * H + 4 * (2 * I // 128) * (H // 128) + M * H + 4 * M * H // 128 + 2 * M * 2 * I) \
+                    + (2 * M * 2 * I + M * I + 4 * M * I // 128) \
+                    + (H * I + 4 * (H // 128) * (I // 128) + M * I + 4 * M * I // 128 + 2 * M * H)
+            else:
+                byts = (2 * M * H + 2 * H + M * H + 4 * M) + gemm_bytes(M, 2 * I, H) \
+                    + (2 * M * 2 * I + M * I + 4 * M) + gemm_bytes(M, H, I)
             gbs = byts / (us * 1e-6) / 1e9
             out["M=%d" % M] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
         else:
@@ -599,7 +615,8 @@ def mlp_chain(dev, g, w8, peak, fp8_peak):
         del x, q1, s1, gu, q2, s2, y
     del Wgu, Wd
     torch.cuda.empty_cache()
-    out["shape"] = "hidden 4096, intermediate 12288, FP8-dynamic; decode frac of the copy peak, prefill of 2 x dense bf16"
+    out["shape"] = "hidden 4096, intermediate 12288, %s; decode frac of the copy peak, prefill of 2 x dense bf16" % (
+        "Block-FP8 (1x128 activation groups, 128x128 weight blocks)" if block else "FP8-dynamic")
     return out
 
 

@@ -1,5 +1,6 @@
 // w8_gemm_grouped.cu -- kernel instantiations: the grouped (mixture-of-experts) form of the
-// Swap-AB GEMM (FP8-dynamic and W8A8-INT8; token tiles of 16, 32 and 64).
+// Swap-AB GEMM (FP8-dynamic and W8A8-INT8; token tiles of 16, 32 and 64 for decode
+// routings, 128 and 256 for prefill routings with hundreds of tokens per expert).
 #include "w8_gemm_kernel.cuh"
 
 namespace w8 {
@@ -20,6 +21,8 @@ cudaError_t launch_bn(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, c
     case 16: return launch_kps<16, KIND>(p, m, a, s);
     case 32: return launch_kps<32, KIND>(p, m, a, s);
     case 64: return launch_kps<64, KIND>(p, m, a, s);
+    case 128: return launch_kps<128, KIND>(p, m, a, s);
+    case 256: return launch_kps<256, KIND>(p, m, a, s);
     default: return cudaErrorNotSupported;
     }
 }

@@ -154,8 +154,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem = *tmem_slot;
     }
 
-    // pair p (the cluster) takes the tiles [p T / P, (p + 1) T / P), weight tile fastest;
-    // with a K split, the K chunk p % S of tile p / S
+    // pair p (the cluster) takes the tiles [p T / P, (p + 1) T / P), weight tile fastest
+    // (token tile fastest, which reads each weight tile from HBM once, measured slower on
+    // B200: 365 against 311 us at M = 4096, K = 4096, N = 24576); with a K split, the K
+    // chunk p % S of tile p / S
     const int P = (int)(gridDim.x >> 1);
     const int pr = (int)(blockIdx.x >> 1);
     const int T = a.tiles;

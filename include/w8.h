@@ -77,10 +77,11 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
 
 /* ---- GEMM variant word -----------------------------------------------------------
  * 0 (W8_VARIANT_AUTO) lets the library choose from its per-shape table (loaded with
- * w8_load_table) or, when the shape is not in it, from a built-in rule: Swap-AB with
- * the balanced partition and a token tile of 16 / 32 / 64 up to 16 / 32 / 64 tokens;
- * past 64 tokens W8_V_PAIR tiles for FP8-dynamic and INT8, and the 64-wide balanced
- * Standard loop for Block-FP8.  An explicit
+ * w8_load_table) or, when the shape is not in it, from a built-in rule: up to 64 tokens
+ * the decode form (W8_V_DECODE, tile and K chunks by a cost model) for FP8-dynamic and
+ * INT8, Swap-AB with the balanced partition and a token tile of 16 / 32 / 64 for
+ * Block-FP8; past 64 tokens W8_V_PAIR tiles for FP8-dynamic and INT8, and the 64-wide
+ * balanced Standard loop for Block-FP8.  An explicit
  * variant sets W8_V_EXPLICIT plus:
  *   W8_V_SWAP_AB  compute out^T = W . Aq^T: the 128-row MMA slot runs over N and the
  *                 narrow slot over tokens (the Swap-AB variant, for small M);
@@ -283,7 +284,8 @@ W8_API int w8_gemm_i32_debug(const void* A_q, const void* W_q, int32_t* acc, int
  * The kernel is the Swap-AB GEMM with the balanced partition: every CTA counts the
  * experts' tiles from the offsets and deals out the units of the experts that have
  * tokens, so empty experts cost nothing.  max_tokens_per_expert (<= T) bounds the tokens
- * of one expert; it picks the token tile (AUTO) and sizes the workspace
+ * of one expert; it picks the token tile (AUTO: 16 / 32 / 64, and past 64 tokens the
+ * 64-token tile with two CTAs per SM) and sizes the workspace
  * (w8_grouped_gemm_workspace_size; same rules as w8_gemm's).  An explicit variant must
  * be Swap-AB with W8_V_STREAM. */
 W8_API int w8_grouped_gemm(int fmt, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,

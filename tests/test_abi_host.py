@@ -135,9 +135,18 @@ def test_variant_resolution_and_workspace(L):
     for fmt in (0, 1):
         assert L.w8_gemm_resolve_variant(fmt, 4096, 4096, 4096, pair) > 0
         assert L.w8_gemm_workspace_size(fmt, 4096, 4096, 4096, pair) == 0
+    # with a K split: one (tile, chunk) unit per pair, so tiles x split <= 74 pairs, and a workspace
+    split4 = w8.variant(False, 4, 256, pair=True)
+    assert L.w8_gemm_resolve_variant(0, 256, 4096, 12288, split4) > 0                 # 16 tiles x 4
+    assert L.w8_gemm_workspace_size(0, 256, 4096, 12288, split4) == 256 * 1024 + 64 * 2 * 256 * 128 * 4
+    assert L.w8_gemm_resolve_variant(0, 256, 4096, 12288, w8.variant(False, 8, 256, pair=True)) == \
+        w8.W8_ERR_UNSUPPORTED                                                            # 16 x 8 > 74
+    assert L.w8_gemm_resolve_variant(0, 256, 4096, 384, w8.variant(False, 4, 256, pair=True)) == \
+        w8.W8_ERR_UNSUPPORTED                                                            # 4 > 3 K blocks
     for fmt, v in ((2, pair), (0, w8.variant(True, 1, 256, pair=True)), (0, w8.variant(False, 2, 256, pair=True)),
                    (0, w8.variant(False, 1, 128, pair=True)), (0, w8.variant(False, 1, 256, stream=True, pair=True)),
                    (0, w8.variant(False, 1, 256, bm64=True, pair=True))):
+        # (the split 2 case: 256 tiles x 2 exceed the pairs)
         assert L.w8_gemm_resolve_variant(fmt, 4096, 4096, 4096, v) == w8.W8_ERR_UNSUPPORTED
     # parallel fixup: 64-row token tile only, no cluster, at most one CTA per SM
     assert L.w8_gemm_resolve_variant(0, 8, 4096, 4096, w8.variant(False, 1, 256, stream=True, bm64=True, pfix=True)) > 0

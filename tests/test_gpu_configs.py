@@ -114,3 +114,47 @@ def test_mlp_chain(orc, mlp, M):
     # the chain's intermediate bf16 may differ in the last bit, which moves a few codes by
     # one step; the end-to-end bound is the GEMM bound
     assert np.max(np.abs(yo - y_ref)) <= TOL_REL * np.max(np.abs(y_ref)) + TOL_ABS
+
+
+@pytest.fixture(scope="module")
+def mlp_block(orc):
+    H, I = 4096, 12288
+    g = synth.gamma(H, seed=synth.SEED_BASE + 6)
+    w_gu = synth.weights(2 * I, H, seed=synth.SEED_BASE + 6 + 1)
+    w_d = synth.weights(H, I, seed=synth.SEED_BASE + 6 + 2)
+    gu_g = w8.w8_quant_weight_block(w_gu.cuda())
+    d_g = w8.w8_quant_weight_block(w_d.cuda())
+    gu_o = orc.quant_weight_block(bits(w_gu))
+    d_o = orc.quant_weight_block(bits(w_d))
+    return H, I, g, gu_g, d_g, gu_o, d_o
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 256, 1024])
+def test_mlp_chain_block_fp8(orc, mlp_block, M):
+    """The MLP block in Block-FP8: rms_norm + 1x128-group quant -> gate_up GEMM (128 x 128
+    weight blocks) -> silu_and_mul + group quant -> down GEMM, AUTO with PDL.  Producer
+    codes and group scales bit for bit on whole sampled rows, the GEMMs within the GEMM
+    bound against the oracle fed with the oracle's own codes."""
+    H, I, g, gu_g, d_g, gu_o, d_o = mlp_block
+    fmt = w8.W8_FMT_BLOCK_FP8
+    x = synth.activations(M, H, seed=synth.SEED_BASE + 6 + 10 * M)
+    xd, gd = x.cuda(), g.cuda()
+    q1, s1 = w8.w8_rmsnorm_quant_group(xd, gd, 1e-6)
+    gu = w8.w8_gemm(fmt, q1, s1, gu_g[0], gu_g[1], variant=AUTO_PDL)
+    q2, s2 = w8.w8_silu_mul_quant_group(gu)
+    y = w8.w8_gemm(fmt, q2, s2, d_g[0], d_g[1], variant=AUTO_PDL)
+    torch.cuda.synchronize()
+    assert np.array_equal(u8(gu_g[0]), gu_o[0]) and np.array_equal(gu_g[1].cpu().numpy(), gu_o[1])
+    rows = list(range(M)) if M <= 8 else sorted(set(np.random.default_rng(M + 1).integers(0, M, 5).tolist()) | {0, M - 1})
+    xr = x[rows].contiguous()
+    oq1, os1 = orc.rmsnorm_quant_group(bits(xr), bits(g), 1e-6)
+    assert np.array_equal(u8(q1)[rows], oq1) and np.array_equal(s1.cpu().numpy()[rows], os1)
+    gu_bits, gu_ref, _ = orc.gemm(2, oq1, os1, gu_o[0], gu_o[1])
+    gu_out = gu.float().cpu().double().numpy()[rows]
+    assert np.max(np.abs(gu_out - gu_ref)) <= TOL_REL * np.max(np.abs(gu_ref)) + TOL_ABS
+    oq2, os2 = orc.silu_mul_quant_group(gu_bits)
+    _, y_ref, _ = orc.gemm(2, oq2, os2, d_o[0], d_o[1])
+    yo = y.float().cpu().double().numpy()[rows]
+    # as in the FP8 chain: a last-bit difference of the intermediate bf16 can move a code
+    assert np.max(np.abs(yo - y_ref)) <= TOL_REL * np.max(np.abs(y_ref)) + TOL_ABS
+    assert w8.w8_device_status(clear=True) == 0

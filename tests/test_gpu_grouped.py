@@ -90,3 +90,17 @@ def test_bad_offsets_compute_nothing(orc):
     torch.cuda.synchronize()
     assert w8.w8_device_status(clear=True) == w8.W8_ERR_INVALID_ARG
     assert torch.all(out == 7.0)
+
+
+PREFILL_ROUTING = [300, 0, 513, 129, 260, 77]
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+@pytest.mark.parametrize("variant", [w8.W8_VARIANT_AUTO, w8.variant(True, 1, 128, stream=True),
+                                     w8.variant(True, 1, 256, stream=True, pdl=True),
+                                     w8.variant(True, 1, 256, stream=True, kps=1)])
+def test_prefill_routing(orc, fmt, variant):
+    """Hundreds of tokens per expert (several 128- or 256-token tiles per expert, ragged
+    last tiles, an empty expert, an expert whose token box must start before its first
+    row near the end of A): the oracle's outputs, untouched rows past the last offset."""
+    run(orc, fmt, PREFILL_ROUTING, 384, 1024, variant=variant, seed=91 + fmt, extra_rows=3)
