@@ -83,6 +83,58 @@ int default_stages(int bn, int kps)
 }  // namespace
 
 // ---------------------------------------------------------------- planning
+// Shared-memory layout of the decode form for q's tile (bn, split, m8, M, kbs; a_region
+// for the fused-quantization form, whose stages carry weights only): the stage count
+// (`stages`, 0 = the default depth), the request padded so that no more CTAs share an SM
+// than its tensor memory holds, and the receive area of the K-split reduction.
+int decode_layout(GemmPlan* q, int stages, bool fq)
+{
+    const int bn = q->bn, C = q->split, M = q->M;
+    const size_t stage = (size_t)((fq ? 0 : q->m8) + bn) * 128;
+    // default depth: about 108 KB of stages and token codes, the most that still lets a CTA
+    // of the next GEMM share the SM (bytes in flight per SM are what sets the streaming rate)
+    if (stages == 0) {
+        const long long room = 110592 - (long long)q->a_region;
+        stages = (int)std::max<long long>(2, std::min<long long>(8, room / (long long)stage));
+    }
+    if (stages < 2) return W8_ERR_UNSUPPORTED;
+    q->stages = stages;
+    // token codes (fq), stages, barriers, TMEM slot and flag, then the scales of the columns
+    // a rank finishes and of the tokens, the ranks' receive-area addresses, and (fq) the
+    // ranks' partial token maxima
+    q->smem_bytes = 1024 + q->a_region + (size_t)stages * stage + (size_t)(2 * stages + 4 + (fq ? 2 : 0)) * 8 + 16 +
+                    (256 + 64 + 8) * 4 + (fq ? (size_t)8 * 64 * 4 : 0);
+    // No more CTAs of this kernel may share an SM than its tensor memory holds: a CTA
+    // waiting for columns another CTA of the same grid holds, while that one waits for
+    // its cluster peers, would stall the grid.  Shared memory (228 KB per SM, 1 KB
+    // reserved per CTA) bounds the CTAs per SM, so pad the request until it does.
+    {
+        const size_t cols = bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
+        const size_t max_ctas = 512 / cols;
+        while (233472 / (q->smem_bytes + 1024) > max_ctas) q->smem_bytes += 1024;
+    }
+    if (q->smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
+    // the partial sums of the columns a rank finishes sit over its stage memory: over the
+    // R stages, for each of the two K-block counts a rank can hold, whose last use comes
+    // earliest (stage s last holds K block s + S floor((n - 1 - s) / S) of n)
+    const size_t recv = (size_t)C * M * (q->sw + 4) * 4;
+    if (recv > (size_t)stages * stage) return W8_ERR_UNSUPPORTED;
+    q->recv_R = (int)((recv + stage - 1) / stage);
+    q->nkb_lo = q->kbs / C;
+    for (int h = 0; h < 2; ++h) {
+        const int n = q->nkb_lo + h;
+        int best = 0x7FFFFFFF;
+        q->recv_first[h] = 0;
+        for (int c0 = 0; c0 + q->recv_R <= stages; ++c0) {
+            int worst = -1;
+            for (int st = c0; st < c0 + q->recv_R; ++st)
+                worst = std::max(worst, st < n ? st + stages * ((n - 1 - st) / stages) : -1);
+            if (worst < best) { best = worst; q->recv_first[h] = c0; }
+        }
+    }
+    return W8_OK;
+}
+
 int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan* p)
 {
     if (M <= 0 || N <= 0 || K <= 0) return W8_ERR_INVALID_ARG;
@@ -107,6 +159,7 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
     q.bm = (variant & W8_V_BM64) ? 64 : 128;
     q.pfix = (variant & W8_V_PFIX) ? 1 : 0;
     if (lg > 8) return W8_ERR_UNSUPPORTED;
+    int rc_layout = W8_OK;
     if (variant & W8_V_DECODE) {
         // decode form (w8_gemm_decode.cu): tokens in the 64-row MMA operand, 16 (tile + 1)
         // weight rows in the wide one, split + 1 K chunks per weight tile as one cluster
@@ -117,50 +170,16 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
         if (bn < 64 || C > 8) return W8_ERR_UNSUPPORTED;
         q.kbs = (K + 127) / 128;
         if (C > q.kbs) return W8_ERR_UNSUPPORTED;
-        // default depth: about 108 KB of stages, the most that still lets a CTA of the next
-        // GEMM share the SM (bytes in flight per SM are what sets the streaming rate)
-        if (stages == 0) stages = (int)std::max<size_t>(2, std::min<size_t>(8, 110592 / ((size_t)(((M + 7) & ~7) + bn) * 128)));
-        if (stages < 2) return W8_ERR_UNSUPPORTED;
         q.decode = 1;
         q.bn = bn;
         q.split = C;
         q.kps = 1;
-        q.stages = stages;
         q.m8 = (M + 7) & ~7;
         q.l2ahead = (variant >> W8_V_L2_SHIFT) & 0xF;
         q.sw = ((bn + 16 * C - 1) / (16 * C)) * 16;
-        const size_t stage = (size_t)(q.m8 + bn) * 128;
-        // stages, barriers, TMEM slot and flag, then the scales of the columns a rank finishes
-        // and of the tokens, and the ranks' receive-area addresses
-        q.smem_bytes = 1024 + (size_t)stages * stage + (size_t)(2 * stages + 4) * 8 + 16 + (256 + 64 + 8) * 4;
-        // No more CTAs of this kernel may share an SM than its tensor memory holds: a CTA
-        // waiting for columns another CTA of the same grid holds, while that one waits for
-        // its cluster peers, would stall the grid.  Shared memory (228 KB per SM, 1 KB
-        // reserved per CTA) bounds the CTAs per SM, so pad the request until it does.
-        {
-            const size_t cols = bn <= 32 ? 32 : bn <= 64 ? 64 : bn <= 128 ? 128 : 256;
-            const size_t max_ctas = 512 / cols;
-            while (233472 / (q.smem_bytes + 1024) > max_ctas) q.smem_bytes += 1024;
-        }
-        if (q.smem_bytes > 232448) return W8_ERR_UNSUPPORTED;
-        // the partial sums of the columns a rank finishes sit over its stage memory: over the
-        // R stages, for each of the two K-block counts a rank can hold, whose last use comes
-        // earliest (stage s last holds K block s + S floor((n - 1 - s) / S) of n)
-        const size_t recv = (size_t)C * M * (q.sw + 4) * 4;
-        if (recv > (size_t)stages * stage) return W8_ERR_UNSUPPORTED;
-        q.recv_R = (int)((recv + stage - 1) / stage);
-        q.nkb_lo = q.kbs / C;
-        for (int h = 0; h < 2; ++h) {
-            const int n = q.nkb_lo + h;
-            int best = 0x7FFFFFFF;
-            q.recv_first[h] = 0;
-            for (int c0 = 0; c0 + q.recv_R <= stages; ++c0) {
-                int worst = -1;
-                for (int st = c0; st < c0 + q.recv_R; ++st)
-                    worst = std::max(worst, st < n ? st + stages * ((n - 1 - st) / stages) : -1);
-                if (worst < best) { best = worst; q.recv_first[h] = c0; }
-            }
-        }
+        q.a_region = 0;
+        rc_layout = decode_layout(&q, stages, false);
+        if (rc_layout != W8_OK) return rc_layout;
         q.nsb = q.kbs;
         q.rows_R = M;
         q.rows_C = N;
@@ -204,9 +223,9 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
         const long long pairs_max = (sm_count > 0 ? sm_count : 148) / 2;
         if (q.split > 1) {
             // one unit per pair, every pair resident at once; a workspace slot of 128 x 256
-            // words per CTA and a ticket counter per half-tile
+            // words per CTA and two counters per half-tile
             const long long units = (long long)q.tiles * q.split;
-            if (units > pairs_max || 2LL * q.tiles > kMaxCounterTiles) return W8_ERR_UNSUPPORTED;
+            if (units > pairs_max || 4LL * q.tiles > kMaxCounterTiles) return W8_ERR_UNSUPPORTED;
             q.G = (int)(2 * units);
             q.align_tiles = 1;
             q.ws_counters = (size_t)kMaxCounterTiles * 4;
@@ -301,6 +320,44 @@ int gemm_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPlan*
 }
 
 // ---------------------------------------------------------------- launch
+namespace {
+// Arguments of the decode-form kernel (plain, or with the quantization fused: then the
+// caller adds x and the debug outputs)
+GemmArgs decode_args(const GemmPlan& p, const float* A_scale, const float* W_scale, void* out, int32_t* out_i32,
+                     int starve, unsigned long long wait_ns)
+{
+    GemmArgs args = {};
+    args.M = p.M; args.N = p.N; args.K = p.K;
+    args.rows_R = p.M; args.rows_C = p.N;
+    args.r_tiles = 1; args.c_tiles = p.c_tiles; args.tiles = p.tiles;
+    args.kbs = p.kbs;
+    args.nsb = p.kbs;
+    args.units = p.units;
+    args.G = p.G;
+    args.align_tiles = 1;
+    args.csplit = p.split;
+    args.stages = p.stages;
+    args.pdl = p.pdl;
+    args.vec_ok = (p.N % 8 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
+    args.sA = A_scale;
+    args.sW = W_scale;
+    args.out = static_cast<__nv_bfloat16*>(out);
+    args.out_i32 = out_i32;
+    args.bn = p.bn;
+    args.m8 = p.m8;
+    args.l2ahead = p.l2ahead;
+    args.sw = p.sw;
+    args.recv_R = p.recv_R;
+    args.nkb_lo = p.nkb_lo;
+    args.recv_first[0] = p.recv_first[0];
+    args.recv_first[1] = p.recv_first[1];
+    args.a_region = (int)p.a_region;
+    args.starve = starve;
+    args.wait_ns = wait_ns;
+    return args;
+}
+}  // namespace
+
 int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const void* W_q, const float* W_scale,
                 void* out, int32_t* out_i32, void* workspace, size_t ws_bytes, cudaStream_t s, const int* g_off,
                 int starve, unsigned long long wait_ns)
@@ -312,33 +369,7 @@ int gemm_launch(const GemmPlan& p, const void* A_q, const float* A_scale, const 
         GemmMaps maps;
         if (!make_tmap(&maps.R, A_q, p.M, p.K, p.m8)) return W8_ERR_CUDA;
         if (!make_tmap(&maps.C, W_q, p.N, p.K, p.bn)) return W8_ERR_CUDA;
-        GemmArgs args = {};
-        args.M = p.M; args.N = p.N; args.K = p.K;
-        args.rows_R = p.M; args.rows_C = p.N;
-        args.r_tiles = 1; args.c_tiles = p.c_tiles; args.tiles = p.tiles;
-        args.kbs = p.kbs;
-        args.nsb = p.kbs;
-        args.units = p.units;
-        args.G = p.G;
-        args.align_tiles = 1;
-        args.csplit = p.split;
-        args.stages = p.stages;
-        args.pdl = p.pdl;
-        args.vec_ok = (p.N % 8 == 0) && ((reinterpret_cast<uintptr_t>(out) & 15) == 0);
-        args.sA = A_scale;
-        args.sW = W_scale;
-        args.out = static_cast<__nv_bfloat16*>(out);
-        args.out_i32 = out_i32;
-        args.bn = p.bn;
-        args.m8 = p.m8;
-        args.l2ahead = p.l2ahead;
-        args.sw = p.sw;
-        args.recv_R = p.recv_R;
-        args.nkb_lo = p.nkb_lo;
-        args.recv_first[0] = p.recv_first[0];
-        args.recv_first[1] = p.recv_first[1];
-        args.starve = starve;
-        args.wait_ns = wait_ns;
+        const GemmArgs args = decode_args(p, A_scale, W_scale, out, out_i32, starve, wait_ns);
         const cudaError_t e = launch_decode(p, maps, args, s);
         if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
         return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
@@ -406,6 +437,21 @@ int linear_plan(int fmt, int M, int N, int K, int variant, int sm_count, GemmPla
     GemmPlan q;
     int rc = gemm_plan(fmt, M, N, K, variant, sm_count, &q);
     if (rc != W8_OK) return rc;
+    if (q.decode) {
+        // decode form: the codes of the rank's K blocks for every token, in a region ahead
+        // of stages that carry weights only (the 64-row MMA reads past the last block's
+        // rows into the stages: rows that are never stored)
+        const int nkb_max = (q.kbs + q.split - 1) / q.split;
+        q.a_region = ((size_t)nkb_max * q.m8 * 128 + 1023) & ~(size_t)1023;
+        // the variant's stage count, or fewer if the code region needs the room
+        int st = (variant >> W8_V_STAGES_SHIFT) & 0xF;
+        rc = decode_layout(&q, st, true);
+        while (rc != W8_OK && st > 2) rc = decode_layout(&q, --st, true);
+        if (rc != W8_OK) return rc;
+        q.fq = 1;
+        *p = q;
+        return W8_OK;
+    }
     // the activations are the narrow C operand of a Swap-AB tile holding every token
     if (!q.swap || q.bm != 128 || q.pfix || q.c_tiles != 1 || q.bn > 64) return W8_ERR_UNSUPPORTED;
     int rg = 0;
@@ -471,6 +517,20 @@ int linear_launch(const GemmPlan& p, const void* x, int ldx, const void* W_q, co
     if (!p.fq) return W8_ERR_INVALID_ARG;
     if (p.ws_bytes > 0 && (workspace == nullptr || ws_bytes < p.ws_bytes)) return W8_ERR_WORKSPACE;
     if (p.ws_bytes > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255)) return W8_ERR_ALIGNMENT;
+    if (p.decode) {
+        // weight boxes only: the kernel reads x and writes the token codes itself
+        GemmMaps maps;
+        if (!make_tmap(&maps.C, W_q, p.N, p.K, p.bn)) return W8_ERR_CUDA;
+        maps.R = maps.C;
+        GemmArgs args = decode_args(p, nullptr, W_scale, out, nullptr, 0, 0);
+        args.x = static_cast<const __nv_bfloat16*>(x);
+        args.ldx = ldx;
+        args.dbg_q = dbg_q;
+        args.dbg_s = dbg_s;
+        const cudaError_t e = launch_decode(p, maps, args, s);
+        if (e == cudaErrorNotSupported) return W8_ERR_UNSUPPORTED;
+        return e == cudaSuccess ? W8_OK : W8_ERR_CUDA;
+    }
     CUtensorMap tR, tX;
     if (!make_tmap(&tR, W_q, p.rows_R, p.K, p.bm)) return W8_ERR_CUDA;
     if (!make_tmap_x(&tX, x, p.M, p.K, ldx, p.fq_m8)) return W8_ERR_CUDA;

@@ -63,31 +63,38 @@ __device__ __forceinline__ void settle_local(uint32_t bar, uint32_t parity)
     while (!ptx::mbar_try_wait(bar, parity) && ptx::globaltimer_ns() - t0 < 10000000ull) {}
 }
 
-template <int KIND>
+template <int KIND, bool FQ>
 __global__ void __launch_bounds__(kThreads, 2)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                        const GemmArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smem_base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int S = a.stages;
     const int BN = a.bn;
     const int m8 = a.m8;
     const int C = a.csplit;
     const int M = a.M;
-    const size_t stage_bytes = (size_t)(m8 + BN) * 128;
+    // FQ: the token codes of this rank's K blocks ([K block][m8 rows][128 bytes], 128-byte
+    // swizzled as a TMA box would land), then stages that carry weight boxes only
+    uint8_t* a_region = smem_base;
+    uint8_t* smem = smem_base + (FQ ? a.a_region : 0);
+    const size_t stage_bytes = (size_t)((FQ ? 0 : m8) + BN) * 128;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)S * stage_bytes);
     uint64_t* empty = full + S;
     uint64_t* tfull = empty + S;     // the accumulator is complete
     uint64_t* freeb = tfull + 1;     // C > 1: the other ranks' MMAs are done (their stages may receive)
     uint64_t* recvb = freeb + 1;     // C > 1: the other ranks' partials of this rank's columns landed
     uint64_t* drain = recvb + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* a_ready = drain + 1;   // FQ: the token codes are in the region
+    uint64_t* amaxb = a_ready + 1;   // FQ, C > 1: the other ranks' partial token maxima landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(FQ ? amaxb + 1 : drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* s_w = reinterpret_cast<float*>(tmem_slot + 4);   // [256] weight scales of this rank's columns
     float* s_a = s_w + 256;                                  // [64] token scales, then [8] words
+    uint32_t* amax_slots = reinterpret_cast<uint32_t*>(s_a + 64 + 8);   // FQ: [8 ranks][64 tokens]
     auto a_slot = [&](int s) { return smem + (size_t)s * stage_bytes; };
-    auto w_slot = [&](int s) { return smem + (size_t)s * stage_bytes + (size_t)m8 * 128; };
+    auto w_slot = [&](int s) { return smem + (size_t)s * stage_bytes + (FQ ? 0 : (size_t)m8 * 128); };
     const int SW = a.sw;
     const int RS = SW + 4;   // row stride in words: token rows fall on different banks
 
@@ -140,10 +147,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         ptx::mbar_init(ptx::smem_u32(freeb), C > 1 ? (uint32_t)(C - 1) : 1u);
         ptx::mbar_init(ptx::smem_u32(recvb), 1);
         ptx::mbar_init(ptx::smem_u32(drain), 1);
+        if (FQ) {
+            ptx::mbar_init(ptx::smem_u32(a_ready), 1);
+            ptx::mbar_init(ptx::smem_u32(amaxb), 1);
+        }
         *abort_flag = 0;
         ptx::fence_barrier_init();
         // the bytes the other ranks will write into this rank's receive area
         if (C > 1) ptx::mbar_arrive_expect_tx(ptx::smem_u32(recvb), (uint32_t)((C - 1) * M * share((int)rank) * 4));
+        // FQ: and their partial token maxima (m8 words each)
+        if (FQ && C > 1) ptx::mbar_arrive_expect_tx(ptx::smem_u32(amaxb), (uint32_t)((C - 1) * m8 * 4));
     }
     if (threadIdx.x == 32) {
         ptx::prefetch_tmap(&tmA);
@@ -184,8 +197,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int first = min(nload, S);   // K blocks whose loads go out without waiting for a stage
             for (int i = first; i < min(nload, first + D); ++i) ptx::tma_prefetch_l2_2d(&tmW, (kb0 + i) * 128, n0);
             ptx::grid_dep_wait();
-            for (int i = 0; i < pre; ++i)
-                ptx::tma_load_2d(ptx::smem_u32(a_slot(i)), &tmA, ptx::smem_u32(full + i), (kb0 + i) * 128, 0, pol_a);
+            if (!FQ)
+                for (int i = 0; i < pre; ++i)
+                    ptx::tma_load_2d(ptx::smem_u32(a_slot(i)), &tmA, ptx::smem_u32(full + i), (kb0 + i) * 128, 0, pol_a);
             int stage = pre % S;
             uint32_t phase = (pre == S) ? 1u : 0u;
             int issued = pre;
@@ -194,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t fb = ptx::smem_u32(full + stage);
                 ptx::mbar_arrive_expect_tx(fb, tx);
                 ptx::tma_load_2d(ptx::smem_u32(w_slot(stage)), &tmW, fb, (kb0 + i) * 128, n0, pol_w);
-                ptx::tma_load_2d(ptx::smem_u32(a_slot(stage)), &tmA, fb, (kb0 + i) * 128, 0, pol_a);
+                if (!FQ) ptx::tma_load_2d(ptx::smem_u32(a_slot(stage)), &tmA, fb, (kb0 + i) * 128, 0, pol_a);
                 if (i >= first && i + D < nload) ptx::tma_prefetch_l2_2d(&tmW, (kb0 + i + D) * 128, n0);
                 ++issued;
                 if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -225,12 +239,14 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint32_t idesc = decode_idesc(KIND, BN);
             int stage = 0;
             uint32_t phase = 0;
-            bool ok = true;
-            for (int i = 0; i < nkb; ++i) {
+            // FQ: the epilogue warps have written the token codes
+            bool ok = !FQ || wait_bounded(ptx::smem_u32(a_ready), 0, abort_flag, wlim);
+            for (int i = 0; i < nkb && ok; ++i) {
                 ok = wait_bounded(ptx::smem_u32(full + stage), phase, abort_flag, wlim);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const uint64_t dA = smem_desc(ptx::smem_u32(a_slot(stage)));
+                const uint64_t dA = FQ ? smem_desc(ptx::smem_u32(a_region + (size_t)i * m8 * 128))
+                                       : smem_desc(ptx::smem_u32(a_slot(stage)));
                 const uint64_t dW = smem_desc(ptx::smem_u32(w_slot(stage)));
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {   // 32 K-bytes per MMA: +2 in 16-byte descriptor units
@@ -273,7 +289,139 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int c = te + j * kEpiThreads;
                 if (c < w && cbase + c < a.N) sw_r[j] = __ldg(a.sW + cbase + c);
             }
-            if (te < M) sa_r = __ldg(a.sA + te);
+            if (!FQ && te < M) sa_r = __ldg(a.sA + te);
+        }
+        if (FQ) {
+            // ---- the activation quantizer, fused: per-token maxima over the row (this
+            // rank's columns, then the other ranks' through distributed shared memory), the
+            // scales, and the codes of this rank's K blocks written where the MMAs read them.
+            // The same scale rule and quotient as the quantizer kernels, so the same codes.
+            constexpr int QF = (KIND == KIND_I8) ? W8_Q_INT8 : W8_Q_FP8;
+            constexpr int kB = 4;   // 16-value chunks per thread with their loads in flight together
+            uint32_t* my_amax = amax_slots + rank * 64;
+            if (te < 64) my_amax[te] = 0u;
+            ptx::bar_sync(kEpiBarrier, kEpiThreads);
+            const int kc0 = kb0 * 128;
+            const int kc1 = min(a.K, (kb0 + nkb) * 128);
+            const int nch = (kc1 - kc0) >> 4;   // 16-value chunks of a token row (K % 16 == 0)
+            const int total = M * nch;          // chunk it: token it / nch, chunk it % nch
+            // a thread's chunks it = te + 128 j; when they all fit in one batch they stay in
+            // registers for the codes, else the codes pass loads them again (from L2)
+            const bool one_batch = total <= kEpiThreads * kB;
+            uint4 xv[2 * kB];
+            auto load_batch = [&](int base) {
+#pragma unroll
+                for (int j = 0; j < kB; ++j) {
+                    const int it = base + j * kEpiThreads;
+                    if (it < total) {
+                        const int mt = it / nch;
+                        const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)mt * a.ldx + kc0 + (it - mt * nch) * 16);
+                        xv[2 * j] = __ldg(src);
+                        xv[2 * j + 1] = __ldg(src + 1);
+                    }
+                }
+            };
+            // the trip count is the same for the 32 lanes of a warp (the warp's first chunk
+            // decides it): the shuffles below need every lane
+            for (int wbase = te - lane; wbase < total; wbase += kEpiThreads * kB) {
+                const int base = wbase + lane;
+                load_batch(base);
+#pragma unroll
+                for (int j = 0; j < kB; ++j) {
+                    const int it = base + j * kEpiThreads;
+                    const int mt = it < total ? it / nch : -1;
+                    float lo[8], hi[8];
+                    unpack_bf16x8(xv[2 * j], lo);
+                    unpack_bf16x8(xv[2 * j + 1], hi);
+                    float mx = 0.0f;   // fmaxf ignores NaN, as the quantizer kernels' maxima do
+                    if (mt >= 0)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fmaxf(fabsf(lo[i]), fabsf(hi[i])));
+                    // one atomic per warp when the warp's 32 chunks belong to one token
+                    const int mt0 = __shfl_sync(0xFFFFFFFFu, mt, 0);
+                    if (__all_sync(0xFFFFFFFFu, mt == mt0)) {
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+                        if (lane == 0 && mt0 >= 0 && mx > 0.0f) atomicMax(my_amax + mt0, __float_as_uint(mx));
+                    } else if (mt >= 0 && mx > 0.0f) {
+                        atomicMax(my_amax + mt, __float_as_uint(mx));   // nonnegative: ordered as integers
+                    }
+                }
+            }
+            ptx::bar_sync(kEpiBarrier, kEpiThreads);
+            bool fq_ok = true;
+            if (C > 1) {
+                // this rank's maxima to every other rank (into the same slot row there)
+                const int pieces = m8 >> 2;
+                if (te < (C - 1) * pieces) {
+                    const int j = te / pieces, pc = te - j * pieces;
+                    const uint32_t r = (uint32_t)(j < (int)rank ? j : j + 1);
+                    const uint4 v = *reinterpret_cast<const uint4*>(my_amax + 4 * pc);
+                    ptx::st_async_v4(ptx::map_to_rank(ptx::smem_u32(my_amax + 4 * pc), r), v.x, v.y, v.z, v.w,
+                                     ptx::map_to_rank(ptx::smem_u32(amaxb), r));
+                }
+                fq_ok = wait_bounded<true>(ptx::smem_u32(amaxb), 0, abort_flag, wlim);
+                if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !fq_ok)) fq_ok = false;
+            }
+            // row maxima, scales and divisors; the row maximum and the divisor's parts are
+            // kept in shared memory once every thread has read the slots
+            uint32_t row_mx = 0u;
+            if (te < M) {
+                for (int r = 0; r < C; ++r) row_mx = max(row_mx, amax_slots[r * 64 + te]);
+                sa_r = scale_from_amax(__uint_as_float(row_mx), QF == W8_Q_FP8 ? kE4M3Max : kInt8Max, false);
+                s_a[te] = sa_r;
+                if (a.dbg_s != nullptr && tile == 0 && rank == 0) a.dbg_s[te] = sa_r;
+            }
+            ptx::bar_sync(kEpiBarrier, kEpiThreads);
+            if (te < M) my_amax[te] = row_mx;
+            ptx::bar_sync(kEpiBarrier, kEpiThreads);
+            // codes of the real chunks
+            auto encode16 = [&](int it, const uint4& v0, const uint4& v1) {
+                const int mt = it / nch, c = it - mt * nch;
+                const int k = kc0 + c * 16;
+                float lo[8], hi[8];
+                unpack_bf16x8(v0, lo);
+                unpack_bf16x8(v1, hi);
+                const RowDivisor d = make_divisor(s_a[mt], __uint_as_float(my_amax[mt]));
+                const uint2 c0 = encode8<QF>(lo, d), c1 = encode8<QF>(hi, d);
+                const uint4 codes = make_uint4(c0.x, c0.y, c1.x, c1.y);
+                const int kbl = c >> 3, c16 = c & 7;
+                *reinterpret_cast<uint4*>(a_region + (size_t)kbl * m8 * 128 + (size_t)mt * 128 +
+                                          (size_t)((c16 ^ (mt & 7)) << 4)) = codes;
+                if (a.dbg_q != nullptr && tile == 0) *reinterpret_cast<uint4*>(a.dbg_q + (size_t)mt * a.K + k) = codes;
+            };
+            if (fq_ok) {
+                for (int base = te; base < total; base += kEpiThreads * kB) {
+                    if (!one_batch) load_batch(base);
+#pragma unroll
+                    for (int j = 0; j < kB; ++j) {
+                        const int it = base + j * kEpiThreads;
+                        if (it < total) encode16(it, xv[2 * j], xv[2 * j + 1]);
+                    }
+                }
+            }
+            // zero codes where no real chunk lands: rows past M, and the columns past K of
+            // the rank's last K block (as the zero-filled box of the two-kernel path)
+            const int pad_rows = m8 - M;
+            const int kpad = nkb * 8 - nch;   // 16-byte chunks past K in the last block
+            for (int it = te; it < pad_rows * nkb * 8 + M * kpad; it += kEpiThreads) {
+                int mt, c;
+                if (it < pad_rows * nkb * 8) {
+                    mt = M + it / (nkb * 8);
+                    c = it - (mt - M) * nkb * 8;
+                } else {
+                    const int r2 = it - pad_rows * nkb * 8;
+                    mt = r2 / kpad;
+                    c = nch + (r2 - mt * kpad);
+                }
+                const int kbl = c >> 3, c16 = c & 7;
+                *reinterpret_cast<uint4*>(a_region + (size_t)kbl * m8 * 128 + (size_t)mt * 128 +
+                                          (size_t)((c16 ^ (mt & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            // the tensor core reads the region through the async proxy
+            ptx::fence_proxy_async_smem();
+            ptx::bar_sync(kEpiBarrier, kEpiThreads);
+            if (te == 0) ptx::mbar_arrive(ptx::smem_u32(a_ready));
         }
         bool ok = wait_bounded(ptx::smem_u32(tfull), 0, abort_flag, wlim);
         if (ptx::bar_red_or(kEpiBarrier, kEpiThreads, !ok)) ok = false;
@@ -434,10 +582,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
-template <int KIND>
+template <int KIND, bool FQ>
 cudaError_t launch_kind(const GemmPlan& p, const GemmMaps& maps, const GemmArgs& args, cudaStream_t s)
 {
-    auto kern = gemm_decode_kernel<KIND>;
+    auto kern = gemm_decode_kernel<KIND, FQ>;
     static bool configured[64] = {};
     static std::mutex mu;
     {
@@ -481,7 +629,9 @@ cudaError_t launch_kind(const GemmPlan& p, const GemmMaps& maps, const GemmArgs&
 cudaError_t launch_decode(const GemmPlan& p, const GemmMaps& m, const GemmArgs& a, cudaStream_t s)
 {
     if (!p.decode || p.swap || p.G % p.split != 0) return cudaErrorNotSupported;
-    return p.fmt == W8_FMT_INT8 ? launch_kind<KIND_I8>(p, m, a, s) : launch_kind<KIND_F8>(p, m, a, s);
+    if (p.fq)
+        return p.fmt == W8_FMT_INT8 ? launch_kind<KIND_I8, true>(p, m, a, s) : launch_kind<KIND_F8, true>(p, m, a, s);
+    return p.fmt == W8_FMT_INT8 ? launch_kind<KIND_I8, false>(p, m, a, s) : launch_kind<KIND_F8, false>(p, m, a, s);
 }
 
 int status_decode(int clear) { return status_word(clear); }

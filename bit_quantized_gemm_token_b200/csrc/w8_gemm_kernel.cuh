@@ -108,6 +108,7 @@ struct GemmArgs {
     int recv_R;           // stages spanned by a rank's receive area
     int nkb_lo;           // the smaller of the two K-block counts a rank holds
     int recv_first[2];    // first stage of the receive area for nkb_lo and nkb_lo + 1 K blocks
+    int a_region;         // with the quantization fused: bytes of the token-code region
     // failure-path check (w8_gemm_timeout_debug): the producer issues no loads and every
     // wait gives up after wait_ns (0: the normal bound)
     int starve;

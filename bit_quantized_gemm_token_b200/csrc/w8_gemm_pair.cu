@@ -17,11 +17,11 @@
 //     leader (remote arrive for rank 1) that the accumulator may be reused.
 // Split-K (split S = 2..8, a power of two): pair p computes K chunk p % S (contiguous K
 // blocks [c kbs / S, (c + 1) kbs / S)) of tile p / S, one unit per pair, so the grid has
-// 2 tiles S CTAs (at most one per SM pair).  Each CTA publishes its 128 x 256 partial
-// sums to its own workspace slot ([column][row] words), takes a ticket on its half-tile's
-// counter, and the last of the S contributors adds the S slots in chunk order -- a fixed
-// order, so results do not depend on which finishes last -- then scales and stores, and
-// resets the counter for the next call.  This fills the chip when a few tall tiles carry
+// 2 tiles S CTAs (at most one per SM pair, all resident at once).  Each CTA publishes its
+// 128 x 256 partial sums to its own workspace slot ([column][row] words) and counts itself
+// in on its half-tile's counter; once all S are in, contributor c adds, for its slice of
+// 256 / S columns, the S slots in chunk order -- a fixed order, so the result does not
+// depend on timing -- then scales and stores; the last to leave resets the counters.  This fills the chip when a few tall tiles carry
 // a long K (the down projection at a few hundred tokens: 16 tiles of K = 12288).
 // Every wait is bounded (1 s, abort flag, device status W8_ERR_DEVICE_TIMEOUT).  No load
 // uses cluster multicast.
@@ -115,7 +115,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* ticket = reinterpret_cast<volatile int*>(tmem_slot + 2);
     auto a_slot = [&](int s) { return smem + (size_t)s * kPairStage; };
     auto b_slot = [&](int s) { return smem + (size_t)s * kPairStage + kHalfBytes; };
 
@@ -296,15 +295,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (++buf == 2) { buf = 0; bphase ^= 1u; }
             if (S_k > 1) {
-                // ticket on this half-tile's counter: the last contributor finishes it
+                // every contributor of the half-tile finishes a column slice once all S have
+                // published (they are all resident: one unit per pair, at most one pair per
+                // two SMs), adding the S partials in chunk order; the last to leave resets
+                // the half-tile's two counters ([arrived, departed]) for the next call
+                int* cnt = a.counters + ((size_t)t * 2 + rank) * 2;
                 __threadfence();
                 ptx::bar_sync(kEpiBarrier, kEpiThreads);
-                if (te == 0) *ticket = atomicAdd(a.counters + t * 2 + (int)rank, 1);
-                ptx::bar_sync(kEpiBarrier, kEpiThreads);
-                if (*ticket == S_k - 1) {
+                bool all_in = true;
+                if (te == 0) {
+                    atomicAdd(cnt, 1);
+                    all_in = wait_count(cnt, S_k, abort_flag);
+                }
+                if (!ptx::bar_red_or(kEpiBarrier, kEpiThreads, !all_in)) {
                     __threadfence();
+                    const int cw = 256 / S_k;   // columns of each contributor's slice
+                    const int cs = chunk * cw;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < 256; c0 += 16) {
+                    for (int c0 = cs; c0 < cs + cw; c0 += 16) {
                         if (c_base + c0 >= a.N) break;
                         uint32_t v[16];
 #pragma unroll
@@ -331,7 +339,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         if (has_row) store_chunk16<KIND, false>(a, a.sA, r_row, c_base + c0, v, s_row);
                     }
-                    if (te == 0) a.counters[t * 2 + (int)rank] = 0;   // ready for the next call
+                    ptx::bar_sync(kEpiBarrier, kEpiThreads);
+                    if (te == 0 && atomicAdd(cnt + 1, 1) == S_k - 1) {
+                        cnt[0] = 0;
+                        cnt[1] = 0;
+                    }
                 }
             }
         }

@@ -58,6 +58,7 @@ struct GemmPlan {
     int recv_R;       // decode: stages spanned by a rank's receive area
     int nkb_lo;       // decode: the smaller of the two K-block counts a rank holds
     int recv_first[2];   // decode: first stage of the receive area for nkb_lo and nkb_lo + 1 K blocks
+    size_t a_region;  // decode with fq: bytes of the token-code region ahead of the stages
     // derived
     int rows_R, rows_C, r_tiles, c_tiles, tiles, kbs;
     int nsb;          // stage blocks (partition units) per tile

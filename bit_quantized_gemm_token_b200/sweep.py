@@ -88,6 +88,9 @@ def candidates(fmt, M, N, K, quick=False, families=("swap", "bm64", "decode")):
     out = []
     if "decode" in families:
         out += decode_candidates(fmt, M, N, K)
+    if "fused" in families and fmt < 2:
+        # the decode form with the activation quantizer inside (w8_linear, one kernel)
+        out += [v | w8.W8_V_FUSED for v in decode_candidates(fmt, M, N, K)]
     if "shipped" in families:
         v = shipped_variant(fmt, M, N, K)
         if v:
@@ -151,7 +154,10 @@ def _legal(fmt, M, N, K, out):
     legal = []
     for v in out:
         try:
-            w8.w8_gemm_resolve_variant(fmt, M, N, K, v)
+            if v & w8.W8_V_FUSED:
+                w8.w8_linear_resolve(fmt, M, N, K, v)
+            else:
+                w8.w8_gemm_resolve_variant(fmt, M, N, K, v)
             legal.append(v)
         except w8.W8Error:
             pass
@@ -195,7 +201,25 @@ class Problem:
         Wq, sW = self.W[copy]
         return w8.w8_gemm(self.fmt, A, sA, Wq, sW, out=out, variant=v, workspace=self.ws)
 
+    def linear(self, M, v, copy=0, out=None):
+        Wq, sW = self.W[copy]
+        return w8.w8_linear(self.fmt, self.X[M], Wq, sW, out=out, variant=v, workspace=self.ws)
+
+    def layer(self, M, v, copy, out):
+        """One layer as used: the activation quantizer and the GEMM, or one kernel."""
+        if v & w8.W8_V_FUSED:
+            self.linear(M, v, copy, out)
+        else:
+            self.quant(M)
+            self.run(M, v, copy, out)
+
     def check(self, M, v, ref_v):
+        if v & w8.W8_V_FUSED:
+            # the fused kernel against the two kernels with the same variant: the same bytes
+            a = self.linear(M, v)
+            b = self.linear(M, v & ~w8.W8_V_FUSED)
+            torch.cuda.synchronize()
+            return torch.equal(a, b)
         A, _ = self.A[M]
         if self.fmt == 1:
             a = w8.w8_gemm_i32_debug(A, self.W[0][0], variant=v, workspace=self.ws)
@@ -222,16 +246,15 @@ def time_in_context(prev, pv, prob, M, v, reps=2):
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     for p, var in ((prev, pv), (prob, v)):
-        p.ws.reserve(w8.w8_gemm_workspace_size(p.fmt, M, p.N, p.K, var))
+        p.ws.reserve(max(w8.w8_gemm_workspace_size(p.fmt, M, p.N, p.K, var & ~w8.W8_V_FUSED),
+                         w8.w8_linear_workspace_size(p.fmt, M, p.N, p.K, var)))
     n = max(prev.ncopy, prob.ncopy)
 
     def body():
         for c in range(n):
-            # as in use: the activation quantizer runs right before every GEMM
-            prev.quant(M)
-            prev.run(M, pv, c % prev.ncopy, prev.out(M))
-            prob.quant(M)
-            prob.run(M, v, c % prob.ncopy, prob.out(M))
+            # as in use: the activation quantizer runs right before every GEMM (or inside it)
+            prev.layer(M, pv, c % prev.ncopy, prev.out(M))
+            prob.layer(M, v, c % prob.ncopy, prob.out(M))
 
     with torch.cuda.stream(s):
         body()
@@ -267,7 +290,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="default pipeline depths only")
     ap.add_argument("--formats", default="0,1,2")
     ap.add_argument("--families", default="swap,bm64,decode",
-                    help="candidate families: swap (Swap-AB), bm64 (64-row token tile), decode, mid (CTA pairs "
+                    help="candidate families: swap (Swap-AB), bm64 (64-row token tile), decode, fused (decode form with "
+                         "the quantizer inside, w8_linear), mid (CTA pairs "
                          "and one-CTA Standard loops for larger token counts), shipped (the current table's "
                          "entry)")
     ap.add_argument("--log", default="")

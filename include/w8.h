@@ -127,10 +127,10 @@ typedef struct CUstream_st* w8_stream_t; /* identical to cudaStream_t */
  *                 Standard loop's sum), no workspace.  split = 2, 4 or 8: one (tile, K
  *                 chunk) unit per pair -- legal only while tiles x split <= SMs / 2 and
  *                 split <= ceil(K / 128) -- each CTA's partial sums go to a workspace
- *                 slot and the last contributor of each half-tile adds the split
- *                 partials in chunk order (a fixed order), scales and stores; workspace
- *                 as for the split partitions (256 KiB of counters, then 256 KiB per
- *                 unit).  Stages default to 5.  INT8 accumulators are exact either way.
+ *                 slot; once all contributors of a half-tile have published, each adds
+ *                 the split partials of its slice of columns in chunk order (a fixed
+ *                 order), scales and stores; workspace as for the split partitions
+ *                 (256 KiB of counters, then 256 KiB per unit).  Stages default to 5.  INT8 accumulators are exact either way.
  *                 With PDL the kernel waits for the kernels ahead before its first load.
  *   W8_V_DECODE   decode form (M <= 64; FP8-dynamic or INT8; no W8_V_SWAP_AB / W8_V_STREAM /
  *                 W8_V_CLUSTER / W8_V_BM64 / W8_V_PAIR): the tokens occupy the tensor
@@ -324,11 +324,14 @@ W8_API int w8_qk_norm_rope(const void* qkv, void* out, int T, int Hq, int Hkv, i
  * inferencia FP8", section "Patron de fusion del forward pass": the quantizer fused
  * into its neighbour; here the neighbour is the GEMM itself.)
  *   When the resolved variant is Swap-AB with every token in one narrow tile (M <= BN
- *   <= 64), ONE kernel does both: each CTA reads x, computes the row (or group) maxima
- *   -- over its own K range, exchanged between the ranks of a cluster split, else over
- *   the whole row -- and writes the codes of the K blocks it multiplies straight into
- *   shared memory, where the tensor core reads them; the quotient x / s is correctly
- *   rounded without a division per element (same codes as the quantizer kernels).
+ *   <= 64), or the decode form (W8_V_DECODE, FP8-dynamic / INT8), ONE kernel can do both:
+ *   each CTA reads x, computes the row (or group) maxima -- over its own K range,
+ *   exchanged between the ranks of a cluster split, else over the whole row -- and
+ *   writes the codes of the K blocks it multiplies straight into shared memory, where
+ *   the tensor core reads them (the decode form: in a code region ahead of weight-only
+ *   stages, written by the epilogue warps while the weights stream); the quotient x / s
+ *   is correctly rounded without a division per element (same codes as the quantizer
+ *   kernels).
  *   Otherwise the quantizer kernel runs first into the workspace, then the GEMM (with
  *   programmatic dependent launch when the variant asks for it).  The one-kernel form is
  *   taken only when requested: an explicit variant carrying W8_V_FUSED (W8_ERR_UNSUPPORTED

@@ -1,5 +1,6 @@
-"""GPU parity of w8_linear, the quantizer fused into the GEMM: the codes and scales the
-kernel computes itself equal the oracle's bit for bit, the outputs equal those of the
+"""GPU parity of w8_linear, the quantizer fused into the GEMM (the Swap-AB form and the
+decode form): the codes and scales the kernel computes itself equal the oracle's bit for
+bit, the outputs equal those of the
 two-kernel path (quantizer, then GEMM) with the same variant bit for bit, and both meet
 the GEMM tolerance against the oracle."""
 import numpy as np
@@ -20,6 +21,12 @@ FUSED = {
     "swap32_stream_pdl": w8.variant(True, 1, 32, stream=True, pdl=True),
     "swap64_split2": w8.variant(True, 2, 64),
     "swap16_cluster8": w8.variant(True, 8, 16, cluster=True, kps=1),
+    # the decode form: the epilogue warps quantize the rank's K blocks into a code region
+    # while the weights stream; row maxima exchanged between the K-chunk ranks
+    "decode_bn256_c1": w8.decode_variant(256, 1),
+    "decode_bn128_c4": w8.decode_variant(128, 4),
+    "decode_bn176_c3_pdl": w8.decode_variant(176, 3, pdl=True),
+    "decode_bn64_c8_st2": w8.decode_variant(64, 8, stages=2),
 }
 
 # (M, N, K): several weight tiles, a ragged last K block (1040), a K range wider than a
