@@ -54,3 +54,21 @@ def test_sweep_candidates_are_legal(fmt, M):
             assert not w8.describe(v)["bm64"]      # the 64-row token tile is FP8 / INT8 only
     ref = sweep.default_variant(fmt, M)
     assert w8.w8_gemm_resolve_variant(fmt, M, N, K, ref) == ref
+
+
+def test_mid_and_fused_families():
+    """Past 64 tokens the sweep offers CTA pairs (whole tiles and K splits that fit one
+    unit per pair) and the one-CTA Standard loops; the fused family offers the decode
+    form with W8_V_FUSED, legal through w8_linear."""
+    K, N = 12288, 4096
+    cands = sweep.candidates(0, 256, N, K, families=("mid",))
+    pairs = [v for v in cands if w8.describe(v)["pair"]]
+    assert pairs and any(w8.describe(v)["split_k"] == 4 for v in pairs)
+    assert not any(w8.describe(v)["split_k"] == 8 for v in pairs)          # 16 tiles x 8 > 74 pairs
+    for v in cands:
+        assert w8.w8_gemm_resolve_variant(0, 256, N, K, v) == v
+    fused = sweep.candidates(0, 8, 4096, 4096, families=("fused",))
+    assert fused and all(v & w8.W8_V_FUSED and v & w8.W8_V_DECODE for v in fused)
+    for v in fused:
+        assert w8.w8_linear_resolve(0, 8, 4096, 4096, v) == v
+    assert sweep.candidates(2, 8, 4096, 5120, families=("fused",)) == []  # no fused decode for Block-FP8
