@@ -296,8 +296,12 @@ def main():
                          "entry)")
     ap.add_argument("--log", default="")
     ap.add_argument("--ms", default=",".join(str(m) for m in MS), help="token counts to sweep")
+    ap.add_argument("--shapes", default="",
+                    help="KxN,KxN,...: sweep these shapes instead of the format's default list (rows of the other "
+                         "shapes are kept); in the layer order they run in")
     args = ap.parse_args()
     ms = [int(m) for m in args.ms.split(",")]
+    only = [tuple(int(v) for v in sh.lower().split("x")) for sh in args.shapes.split(",")] if args.shapes else None
     families = tuple(args.families.split(","))
     # rows of formats not swept now are kept from the table being replaced
     kept = []
@@ -307,7 +311,10 @@ def main():
     if os.path.exists(args.out):
         for line in open(args.out):
             f = line.split("#")[0].split()
-            if len(f) == 5 and (int(f[0]) not in fmts_swept or int(f[3]) not in ms):
+            if len(f) != 5:
+                continue
+            swept_shape = only is None or (int(f[2]), int(f[1])) in only
+            if int(f[0]) not in fmts_swept or int(f[3]) not in ms or not swept_shape:
                 kept.append((int(f[0]), int(f[1]), int(f[2]), int(f[3]), int(f[4], 16)))
     os.environ["W8_TABLE"] = "none"
     w8.w8_clear_table()
@@ -319,7 +326,7 @@ def main():
     t_start = time.time()
     top_n = 8
     for fmt in fmts:
-        shapes = BLOCK if fmt >= 2 else DENSE
+        shapes = only if only else (BLOCK if fmt >= 2 else DENSE)
         probs = [Problem(fmt, N, K, ms, dev) for (K, N) in shapes]
         for M in ms:
             ref_v = default_variant(fmt, M)
