@@ -88,26 +88,61 @@ __device__ __forceinline__ DSum block_sum_dd(DSum v, DSum* red)
 // ln2 split into a short leading part and a remainder, exp(r) by its Taylor series to
 // degree 7 (Horner, fused multiply-adds), and the exact scaling by 2^n as two
 // power-of-two factors that stay normal.  Each step is an explicitly rounded fp32 op,
-// so the result is fully specified (worst error about 1 ulp against exp).
-__device__ __forceinline__ float exp_cw(float x)
+// so the result is fully specified (worst error about 1 ulp against exp).  It is computed
+// for two values at once (exp_cw2 below).
+
+// Two fp32 values in one 64-bit register, for the paired fp32 instructions of sm_100
+// (fma.rn.f32x2 / mul.rn.f32x2: each half an independent, correctly rounded operation)
+__device__ __forceinline__ unsigned long long f2pack(float a, float b)
 {
-    if (x != x) return x;
-    if (x > 100.0f) return __int_as_float(0x7F800000);
-    if (x < -150.0f) return 0.0f;
-    const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));   // log2(e)
-    float r = __fmaf_rn(-n, 0x1.62e400p-1f, x);             // ln 2, leading bits
-    r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);                  // ln 2, remainder
-    float p = 0x1.a01a02p-13f;                              // 1/7!
-    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                   // 1/6!
-    p = __fmaf_rn(p, r, 0x1.111112p-7f);                    // 1/5!
-    p = __fmaf_rn(p, r, 0x1.555556p-5f);                    // 1/4!
-    p = __fmaf_rn(p, r, 0x1.555556p-3f);                    // 1/3!
-    p = __fmaf_rn(p, r, 0.5f);
-    p = __fmaf_rn(p, r, 1.0f);
-    p = __fmaf_rn(p, r, 1.0f);
-    const int ni = static_cast<int>(n);
-    const int n1 = ni / 2, n2 = ni - n1;
-    return __fmul_rn(__fmul_rn(p, __int_as_float((n1 + 127) << 23)), __int_as_float((n2 + 127) << 23));
+    return ((unsigned long long)__float_as_uint(b) << 32) | __float_as_uint(a);
+}
+__device__ __forceinline__ float f2lo(unsigned long long v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(unsigned long long v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The exp described above, for two values at once: each gets the same sequence of
+// correctly rounded operations, paired (half the instructions for the reduction, the
+// polynomial and the scaling; 115 -> 109 us for silu_and_mul + quant at 4096 x 12288 on
+// B200).  NaN gives
+// NaN, x > 100 gives +inf and x < -150 gives 0; those inputs run the normal path on a
+// clamped value first.
+__device__ __forceinline__ void exp_cw2(float x0, float x1, float& e0, float& e1)
+{
+    const float c0 = fminf(fmaxf(x0, -150.0f), 100.0f), c1 = fminf(fmaxf(x1, -150.0f), 100.0f);
+    const unsigned long long X = f2pack(c0, c1);
+    const unsigned long long T = mul2(X, f2pack(0x1.715476p+0f, 0x1.715476p+0f));   // log2(e)
+    const float n0 = rintf(f2lo(T)), n1 = rintf(f2hi(T));
+    const unsigned long long NN = f2pack(-n0, -n1);
+    unsigned long long R = fma2(NN, f2pack(0x1.62e400p-1f, 0x1.62e400p-1f), X);     // ln 2, leading bits
+    R = fma2(NN, f2pack(0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f), R);                      // ln 2, remainder
+    unsigned long long P = f2pack(0x1.a01a02p-13f, 0x1.a01a02p-13f);                // 1/7!
+    P = fma2(P, R, f2pack(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
+    P = fma2(P, R, f2pack(0x1.111112p-7f, 0x1.111112p-7f));
+    P = fma2(P, R, f2pack(0x1.555556p-5f, 0x1.555556p-5f));
+    P = fma2(P, R, f2pack(0x1.555556p-3f, 0x1.555556p-3f));
+    P = fma2(P, R, f2pack(0.5f, 0.5f));
+    P = fma2(P, R, f2pack(1.0f, 1.0f));
+    P = fma2(P, R, f2pack(1.0f, 1.0f));
+    const int i0 = (int)n0, i1 = (int)n1;
+    const int a0 = i0 / 2, a1 = i1 / 2;
+    P = mul2(P, f2pack(__int_as_float((a0 + 127) << 23), __int_as_float((a1 + 127) << 23)));
+    P = mul2(P, f2pack(__int_as_float((i0 - a0 + 127) << 23), __int_as_float((i1 - a1 + 127) << 23)));
+    e0 = f2lo(P);
+    e1 = f2hi(P);
+    if (x0 != x0) e0 = x0; else if (x0 > 100.0f) e0 = __int_as_float(0x7F800000); else if (x0 < -150.0f) e0 = 0.0f;
+    if (x1 != x1) e1 = x1; else if (x1 > 100.0f) e1 = __int_as_float(0x7F800000); else if (x1 < -150.0f) e1 = 0.0f;
 }
 
 // Grouped (1x128) variant of the last step of the row kernels: the 16 chunks of a
@@ -366,10 +401,12 @@ __device__ __forceinline__ void silu_row(const uint4 (&rg)[CPT], const uint4 (&r
             unpack_bf16x8(rg[c], g);
             unpack_bf16x8(ru[c], u);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float den = __fadd_rn(1.0f, exp_cw(-g[i]));
-                h[c][i] = __fmul_rn(__fdiv_rn(g[i], den), u[i]);
-                amax = fmaxf(amax, fabsf(h[c][i]));
+            for (int i = 0; i < 8; i += 2) {
+                float e0, e1;
+                exp_cw2(-g[i], -g[i + 1], e0, e1);
+                h[c][i] = __fmul_rn(__fdiv_rn(g[i], __fadd_rn(1.0f, e0)), u[i]);
+                h[c][i + 1] = __fmul_rn(__fdiv_rn(g[i + 1], __fadd_rn(1.0f, e1)), u[i + 1]);
+                amax = fmaxf(amax, fmaxf(fabsf(h[c][i]), fabsf(h[c][i + 1])));
             }
         }
     }
