@@ -116,13 +116,29 @@ __device__ __forceinline__ float quotient_plain(float x, const RowDivisor& d)
 }
 
 // 8 values / s -> 8 codes packed little-endian into a uint2 (d = make_divisor(s)).
+// quotient_plain of two values at once on the paired fp32 instructions of sm_100
+// (fma.rn.f32x2 / mul.rn.f32x2: each half the same correctly rounded operation, so each
+// quotient equals quotient_plain's)
+__device__ __forceinline__ void quotient_plain2(float x0, float x1, const RowDivisor& d, float& q0, float& q1)
+{
+    const unsigned long long X = ((unsigned long long)__float_as_uint(x1) << 32) | __float_as_uint(x0);
+    const unsigned long long Y = ((unsigned long long)__float_as_uint(d.y) << 32) | __float_as_uint(d.y);
+    const unsigned long long NS = ((unsigned long long)__float_as_uint(-d.s) << 32) | __float_as_uint(-d.s);
+    unsigned long long Q, R, Z;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(Q) : "l"(X), "l"(Y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(R) : "l"(Q), "l"(NS), "l"(X));   // x - q0 s', exact
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Z) : "l"(R), "l"(Y), "l"(Q));
+    q0 = copysignf(__uint_as_float((uint32_t)Z), x0);
+    q1 = copysignf(__uint_as_float((uint32_t)(Z >> 32)), x1);
+}
+
 template <int QFMT>
 __device__ __forceinline__ uint2 encode8(const float (&f)[8], const RowDivisor& d)
 {
     float v[8];
     if (d.plain) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = quotient_plain(f[i], d);
+        for (int i = 0; i < 8; i += 2) quotient_plain2(f[i], f[i + 1], d, v[i], v[i + 1]);
     } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) v[i] = quotient_rn(f[i], d);

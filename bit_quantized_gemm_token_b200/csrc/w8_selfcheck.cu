@@ -4,7 +4,7 @@
 // The codes are defined from the correctly rounded quotient x / s; the kernels multiply
 // by a prepared reciprocal and correct the result with one fused multiply-add
 // (Markstein's method; the shorter plain form where no scaling is needed and the row's
-// maximum is finite).  The two must give the same 8-bit code for every input a
+// maximum is finite, one value at a time and paired on the f32x2 instructions).  The two must give the same 8-bit code for every input a
 // quantizer can meet, and the same fp32 quotient wherever a code can depend on it
 // (|x / s| >= 2^-10).
 //   modes 0, 1, 2 (bf16 numerators: the plain quantizers): every bf16 amax from the
@@ -31,14 +31,23 @@ __device__ __forceinline__ void compare(int rule, float amax, float s, const Row
 {
     const float q1 = __fdiv_rn(x, s);
     const float q2 = quotient_rn(x, d);
-    // the plain form wherever the quantizers take it (no scaling, finite amax)
-    const float q3 = d.plain ? quotient_plain(x, d) : q2;
+    // the plain form wherever the quantizers take it (no scaling, finite amax), scalar and
+    // paired (with -x beside x)
+    float q3 = q2;
+    bool pair_bad = false;   // the paired form differs from the scalar one in any bit
+    if (d.plain) {
+        q3 = quotient_plain(x, d);
+        float p0, p1;
+        quotient_plain2(x, -x, d, p0, p1);
+        pair_bad = __float_as_uint(p0) != __float_as_uint(q3) ||
+                   __float_as_uint(p1) != __float_as_uint(quotient_plain(-x, d));
+    }
     const uint32_t c1 = rule == 1 ? int8_code(q1) : (e4m3x2(q1, 0.0f) & 0xFFu);
     const uint32_t c2 = rule == 1 ? int8_code(q2) : (e4m3x2(q2, 0.0f) & 0xFFu);
     const uint32_t c3 = rule == 1 ? int8_code(q3) : (e4m3x2(q3, 0.0f) & 0xFFu);
     // the quotient must match wherever a code can depend on it: |x / s| >= 2^-10
     const bool coded = fabsf(q1) >= 0x1p-10f && isfinite(q1);
-    if (c1 != c2 || c1 != c3 ||
+    if (pair_bad || c1 != c2 || c1 != c3 ||
         (coded && (__float_as_uint(q1) != __float_as_uint(q2) || __float_as_uint(q1) != __float_as_uint(q3)))) {
         ++bad;
         fa = abits;
